@@ -1,0 +1,440 @@
+#!/usr/bin/env python
+"""Benchmark of the attention core: global attention over S=100 frames x 1031
+tokens (103,100 tokens, 16 heads x 64, bf16), the headline workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+One step = one vggt_attn_global call (QK-LayerNorm + RoPE prologue, then the
+tcgen05 attention core) on inputs resident in HBM.  `value` is the
+algorithmic TFLOP/s (4 * N^2 * 64 * H per call: QK^T and PV only) summed over
+all ranks, from CUDA-event time (max over ranks).  Side measurements in the
+same run: `e2e` (the same call with pinned host buffers, H2D + D2H inside the
+timed region), `roofline` (the core kernel alone against the measured bf16
+peak), `modes` (ms per mode on the other workloads), `clocks` (nvidia-smi
+sampled during the timed region) and `cpu_baseline` (the fp64 oracle on a
+bounded sample, on this host's cores).
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own,
+independent copy of the workload (an independent scene), so per-GPU work is
+fixed and no data crosses ranks ("scaling": "weak").  `--impl reference` runs
+the fp64 oracle instead (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+HEADLINE = 3                      # global, S=100, 103,100 tokens, H=16
+METRIC = "global-attn TFLOP/s & % bf16 tensor peak (S=100, 103k tok); ms/layer per mode"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+CORE_SRC = os.path.join(ROOT, "vit_attention_b200", "csrc", "attention_sm100.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_core_global_S100_traffic.txt")
+
+
+def attention_flops(mode: str, shape) -> float:
+    """Algorithmic flops of one call: 4 * Nq * Nk * 64 per head (QK^T + PV)."""
+    if mode == "global":
+        n = shape.S * shape.T
+        return 4.0 * n * n * 64 * shape.H
+    if mode == "frame":
+        return 4.0 * shape.S * shape.T * shape.T * 64 * shape.H
+    n = shape.S * shape.n_special
+    return 4.0 * n * n * 64 * shape.H
+
+
+def io_bytes(mode: str, shape) -> float:
+    """Minimum HBM bytes of one call: read the q/k/v it uses, write its output rows."""
+    rows = shape.S * (shape.n_special if mode == "register" else shape.T)
+    return rows * shape.H * 64 * 2 * 4.0
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    return int(os.environ.get("RANK", "0")), int(os.environ.get("WORLD_SIZE", "1")), \
+        int(os.environ.get("LOCAL_RANK", "0"))
+
+
+def shard_plan(world: int, rank: int, base_seed: int):
+    """Weak scaling: rank r runs one independent copy of the workload (its own seed)."""
+    return {"rank": rank, "world": world, "seed": base_seed + 7919 * rank, "problems": 1}
+
+
+def reduce_max(value: float, device=None) -> float:
+    """Max of a scalar over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.hw_slowdown",
+              "clocks_event_reasons.hw_thermal_slowdown", "clocks_event_reasons.sw_thermal_slowdown",
+              "clocks_event_reasons.sw_power_cap", "utilization.gpu"]
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.lines = []
+        self.gpu_id = None
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            self.gpu_id = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.gpu_id = str(device_index)
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, "--query-gpu=" + ",".join(self.FIELDS),
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        samples = []
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != len(self.FIELDS):
+                continue
+            try:
+                samples.append({"sm": float(parts[0]), "max": float(parts[1]), "power": float(parts[2]),
+                                "hw": parts[3], "hwt": parts[4], "swt": parts[5], "pcap": parts[6],
+                                "util": float(parts[7])})
+            except ValueError:
+                continue
+        if not samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        loaded = [s for s in samples if s["util"] >= 50] or samples
+        reasons = set()
+        for s in loaded:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if s[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(s["sm"] for s in loaded), "sm_max_mhz": max(s["max"] for s in loaded),
+                "reasons": sorted(reasons), "samples": len(loaded),
+                "power_w_max": max(s["power"] for s in loaded)}
+
+
+# ---------------------------------------------------------------- helpers
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def core_source_hash() -> str:
+    with open(CORE_SRC, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per launch of the core kernel from the committed ncu summary,
+    or None when absent or taken on a different kernel source."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    text = open(TRAFFIC_FILE).read()
+    m_b = re.search(r"dram_bytes_per_launch\s*=\s*([0-9.eE+]+)", text)
+    m_h = re.search(r"kernel_source_sha256_16\s*=\s*([0-9a-f]+)", text)
+    if not m_b or not m_h or m_h.group(1) != core_source_hash():
+        return None
+    return float(m_b.group(1))
+
+
+def device_inputs(x, device):
+    import torch
+    qkv = torch.from_numpy(x["qkv"].view(np.int16)).to(device).view(torch.bfloat16)
+    prm = {k: torch.from_numpy(np.ascontiguousarray(x[k])).to(device)
+           for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}
+    return qkv, prm
+
+
+def cuda_time_ms(fn, stream, iters: int) -> float:
+    """Average ms per call of fn() over `iters` calls, CUDA events on `stream`."""
+    import torch
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    start.record(stream)
+    for _ in range(iters):
+        fn()
+    end.record(stream)
+    end.synchronize()
+    return start.elapsed_time(end) / iters
+
+
+# ---------------------------------------------------------------- oracle (CPU baseline / reference arm)
+def oracle_sample(workload, n_queries: int, seed: int = 0):
+    """Time the fp64 oracle on `n_queries` seeded queries of `workload` (global mode).
+
+    Returns (seconds, algorithmic flops of the sample, threads used)."""
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    x = W.make_inputs(workload)
+    shape = workload.shape
+    q = W.query_subset(shape.S * shape.T, n_queries, workload.seed + seed)
+    t0 = time.perf_counter()
+    O.attn_global(shape, x, q)
+    dt = time.perf_counter() - t0
+    n = shape.S * shape.T
+    flops = 4.0 * n_queries * n * 64 * shape.H
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return dt, flops, threads
+
+
+def cpu_baseline(n_queries: int):
+    w = W.workload(HEADLINE)
+    dt, flops, threads = oracle_sample(w, n_queries)
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"fp64 numpy oracle, global mode, {n_queries} seeded queries x all 16 heads over all "
+                      f"{w.shape.S * w.shape.T} keys (incl. LN+RoPE of every key), {dt:.1f} s",
+            "seconds": dt}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = W.workload(HEADLINE)
+    n_q = args.ref_queries
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt, flops, threads = oracle_sample(w, n_q, seed=i)
+        if i >= args.warmup:
+            times.append(dt)
+    value = flops / statistics.mean(times) / 1e12
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": w.name, "tokens": w.shape.S * w.shape.T, "heads": 16,
+                                            "head_dim": 64, "sample_queries_per_step": n_q},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                             "sample": f"{n_q} seeded queries x 16 heads over all keys per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+def run_ours(args):
+    import torch
+    import torch.distributed as dist
+    import datetime
+
+    import vit_attention_b200 as V
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+
+    w = W.workload(HEADLINE)
+    shape = w.shape
+    plan = shard_plan(world, rank, w.seed)
+    x = W.make_random_inputs(shape, plan["seed"], w.lowrank) if rank else W.make_inputs(w)
+    qkv, prm = device_inputs(x, device)
+    out = torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device=device)
+    ws_bytes = V.vggt_attn_workspace_size(shape, "global")
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device)
+    flops = attention_flops("global", shape)
+
+    def step():
+        V.vggt_attn_global(shape, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"], prm["k_beta"], out, ws,
+                           ws_bytes, stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert V.vggt_attn_read_status(ws, stream) == 0
+
+    # ---- timed region: K steps, barrier + synchronize on both sides, max over ranks
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    time.sleep(0.4)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for _ in range(args.steps):
+        step()
+    end.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clk = clocks.stop()
+    ms_local = start.elapsed_time(end)
+    ms = reduce_max(ms_local, device)
+    status = V.vggt_attn_read_status(ws, stream)
+    if status != 0:
+        raise RuntimeError(f"device status {status} ({V.error_string(status)})")
+    value = flops * args.steps * world / (ms / 1000.0) / 1e12
+    launches = 2 * args.steps      # prologue + core per call
+
+    # ---- roofline: the core kernel alone (CUDA events on its stream)
+    peaks, peak_src = load_peaks()
+    core_ms = cuda_time_ms(lambda: V.vggt_attn_core("global", shape, qkv, out, ws, ws_bytes, stream), stream,
+                           max(3, args.steps))
+    pro_ms = cuda_time_ms(lambda: V.vggt_attn_prologue("global", shape, qkv, prm["q_gamma"], prm["q_beta"],
+                                                       prm["k_gamma"], prm["k_beta"], ws, ws_bytes, stream),
+                          stream, 10)
+    core_tflops = flops / (core_ms / 1000.0) / 1e12
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    traffic = recorded_traffic()
+    roofline = {"bound": "tensor", "achieved": core_tflops, "peak": peak, "unit": "TFLOP/s",
+                "frac": core_tflops / peak, "traffic": traffic,
+                "kernel": "vggt::attn_core_kernel", "kernel_ms": core_ms,
+                "peak_source": f"{peak_src} bf16_tflops_sustained (back-to-back launches, seconds long)",
+                "frac_of_burst_peak": core_tflops / peaks.get("bf16_tflops", peak),
+                "prologue_ms": pro_ms,
+                "prologue_hbm_gbs": (shape.S * shape.T * shape.H * 64 * 2 * 4) / (pro_ms / 1000) / 1e9}
+
+    # ---- e2e: same call from pinned host buffers, H2D + D2H inside the timed region
+    h_qkv = torch.empty(qkv.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_qkv.copy_(qkv)
+    h_prm = {k: v.cpu().pin_memory() for k, v in prm.items()}
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    d_qkv = torch.empty_like(qkv)
+    d_prm = {k: torch.empty_like(v) for k, v in prm.items()}
+
+    def e2e_step():
+        d_qkv.copy_(h_qkv, non_blocking=True)
+        for k in d_prm:
+            d_prm[k].copy_(h_prm[k], non_blocking=True)
+        V.vggt_attn_global(shape, d_qkv, d_prm["q_gamma"], d_prm["q_beta"], d_prm["k_gamma"], d_prm["k_beta"], out,
+                           ws, ws_bytes, stream)
+        h_out.copy_(out, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    e2e_iters = max(3, min(args.steps, 10))
+    barrier(device)
+    e2e_ms = reduce_max(cuda_time_ms(e2e_step, stream, e2e_iters), device)
+    h2d = qkv.numel() * 2 + sum(v.numel() * 4 for v in prm.values())
+    d2h = out.numel() * 2
+    e2e = {"value": flops * world / (e2e_ms / 1000.0) / 1e12, "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del h_qkv, h_out, d_qkv
+
+    # ---- ms/layer per mode on the other workloads (device-drawn inputs of the same shapes)
+    modes = {}
+    if not args.no_modes:
+        modes = mode_timings(V, device, stream)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.cpu_queries)
+
+    if world > 1:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "mode": "global", "frames": shape.S, "tokens": shape.S * shape.T,
+                       "heads": shape.H, "head_dim": 64, "flops_per_step_per_gpu": flops,
+                       "l2": "no flush: qkv 633 MB + workspace 422 MB per step exceed the 126 MB L2",
+                       "parallelism": f"independent replicas x{world} (weak)"},
+            "pct_of_peak": 100.0 * value / world / peak,
+            "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
+            "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def mode_timings(V, device, stream):
+    """ms per call for each mode on its workload, plus the S=500 layer (register + frame)."""
+    import torch
+    res = {}
+    g = torch.Generator(device=device)
+    g.manual_seed(1234)
+    for label, idx, mode in (("frame_S24_T1031", 1, "frame"), ("global_S24_N24744", 2, "global"),
+                             ("register_S500", 4, "register"), ("frame_S500", 4, "frame")):
+        shape = W.workload(idx).shape
+        if label == "frame_S500":
+            pass  # reuses the S=500 tensors of the register entry
+        else:
+            qkv = torch.randn((shape.S, shape.T, 3, shape.H, 64), generator=g, device=device,
+                              dtype=torch.float32).to(torch.bfloat16)
+            prm = {k: (1.0 if "gamma" in k else 0.0) + 0.1 * torch.randn((shape.H, 64), generator=g, device=device)
+                   for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}
+            out = torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device=device)
+        wsb = V.vggt_attn_workspace_size(shape, mode)
+        ws = torch.empty(wsb, dtype=torch.uint8, device=device)
+        fn = lambda: V.attend(mode, shape, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"], prm["k_beta"], out,
+                              ws, stream)
+        for _ in range(3):
+            fn()
+        ms = cuda_time_ms(fn, stream, 10)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        f = attention_flops(mode, shape)
+        res[label] = {"ms": ms, "tflops": f / (ms / 1000) / 1e12, "gbs_min_io": io_bytes(mode, shape) / (ms / 1000) / 1e9}
+        del ws
+    res["layer_S500_register_plus_frame_ms"] = res["register_S500"]["ms"] + res["frame_S500"]["ms"]
+    return res
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-queries", type=int, default=24, help="oracle sample size of the CPU baseline")
+    ap.add_argument("--ref-queries", type=int, default=8, help="oracle queries per step of --impl reference")
+    ap.add_argument("--no-modes", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_ours(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

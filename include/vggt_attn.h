@@ -1,0 +1,154 @@
+/*
+ * vggt_attn.h -- C ABI of libvggt_attn.so, the sm_100a (B200) attention core
+ * of a VGGT-style alternating-attention block.
+ *
+ * What it computes (VGGT-Omega Aggregator explainer, sections 2 and 3):
+ * for every token and head, q and k go through a LayerNorm over the 64 head
+ * dimensions with a per-head affine ("use_qk_norm=True"), patch tokens are
+ * rotated by a 2D rotary position embedding from their (row, col) in the
+ * patch grid (re-applied at every layer; HTTM article, "04 method"), and then
+ * exact softmax attention runs in one of three modes:
+ *   frame    -- each frame's T tokens attend among themselves (section 3, step 1);
+ *   global   -- all S*T tokens form one sequence (section 3, mode 1);
+ *   register -- only the n_special camera + register tokens of every frame
+ *               attend, over each other (section 3, mode 2).
+ *
+ * Conventions fixed by this library where the pages are silent:
+ *   - LayerNorm: biased variance, epsilon = shape->ln_eps (> 0).
+ *   - RoPE: dims [0,32) rotate by the patch row, [32,64) by the patch column;
+ *     within each 32-dim half, pair (j, j+16), j in [0,16), rotates by angle
+ *     pos * rope_base^(-2j/32), (a, b) -> (a cos - b sin, b cos + a sin).
+ *     Token t >= n_special is patch p = t - n_special at row p / grid_w,
+ *     col p % grid_w (0-based); tokens t < n_special are not rotated.  Every
+ *     frame uses the same positions, in global mode too.
+ *   - softmax scale: shape->softmax_scale, or 1/sqrt(64) when <= 0.
+ *   - register mode writes only rows t < n_special of every frame of `out`;
+ *     patch rows are left byte-for-byte untouched.
+ *
+ * Data layout (all device memory, caller-owned, row-major, no padding):
+ *   qkv      bf16 [S][T][3][H][64]   (index 0 = q, 1 = k, 2 = v), 16-byte aligned
+ *   q_gamma, q_beta, k_gamma, k_beta   fp32 [H][64], 16-byte aligned
+ *   out      bf16 [S][T][H][64], 16-byte aligned, must not overlap qkv
+ *   workspace  >= vggt_attn_workspace_size(shape, mode) bytes, 256-byte aligned;
+ *              holds the normalised, rotated bf16 q and k (and, in register
+ *              mode, the gathered v) plus a status word.  Its contents
+ *              between calls are the library's; one workspace must not be used
+ *              by two calls that may run concurrently.
+ *
+ * Numerics: q and k are normalised and rotated in fp32, then rounded to bf16
+ * (q pre-multiplied by softmax_scale * log2(e)); scores accumulate in fp32 on
+ * the tensor cores; the online softmax runs in fp32 with base-2 exponentials;
+ * probabilities are rounded to bf16 for the P.V product (fp32 accumulate); the
+ * output is rounded to bf16 (nearest even).
+ *
+ * Calls are asynchronous: they validate every argument on the host, enqueue
+ * kernels on `cuda_stream` (a cudaStream_t; NULL = legacy default stream) and
+ * return without synchronising.  They allocate nothing.  Argument errors are
+ * reported before anything is enqueued, with no side effects.  A device-side
+ * failure (a bounded wait inside a kernel that ran out) is recorded in the
+ * workspace status word and read with vggt_attn_read_status().
+ *
+ * Thread safety: no mutable global state; concurrent calls on different
+ * workspaces are safe.
+ */
+#ifndef VGGT_ATTN_H
+#define VGGT_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define VGGT_ATTN_ABI_VERSION 1
+
+/* Return codes (0 = success). */
+enum {
+  VGGT_ATTN_OK = 0,
+  VGGT_ATTN_ERR_INVALID_ARG = -1,       /* NULL pointer, bad mode, overlapping buffers, non-finite scalar */
+  VGGT_ATTN_ERR_UNSUPPORTED_SHAPE = -2, /* head_dim != 64, T != n_special + grid_h*grid_w, sizes out of range */
+  VGGT_ATTN_ERR_MISALIGNED = -3,        /* a pointer lacks the alignment stated above */
+  VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL = -4,
+  VGGT_ATTN_ERR_CUDA = -5,              /* a CUDA runtime/driver call or a launch failed */
+  VGGT_ATTN_ERR_TIMEOUT = -6,           /* a bounded wait inside a kernel expired (vggt_attn_read_status) */
+  VGGT_ATTN_ERR_UNSUPPORTED_DEVICE = -7 /* current device is not compute capability 10.0 (sm_100a) */
+};
+
+/* Attention modes. */
+enum { VGGT_ATTN_FRAME = 0, VGGT_ATTN_GLOBAL = 1, VGGT_ATTN_REGISTER = 2 };
+
+typedef struct {
+  int S;               /* frames, >= 1 */
+  int T;               /* tokens per frame, >= 1 */
+  int H;               /* heads, >= 1 */
+  int head_dim;        /* must be 64 */
+  int n_special;       /* camera + register tokens at the start of every frame, 0..T (>= 1 for register mode) */
+  int grid_h, grid_w;  /* patch grid; T == n_special + grid_h * grid_w */
+  float ln_eps;        /* QK-LayerNorm epsilon, > 0 */
+  float rope_base;     /* RoPE base (100 for the VGGT-style aggregator), > 0 */
+  float softmax_scale; /* <= 0 selects 1/sqrt(head_dim) */
+} vggt_attn_shape;
+
+/* Bytes of workspace a call in `mode` needs for `shape`; 0 if the shape or
+ * mode is invalid. */
+size_t vggt_attn_workspace_size(const vggt_attn_shape* shape, int mode);
+
+/* Frame mode: each frame's tokens attend within the frame.  Writes all of `out`. */
+int vggt_attn_frame(const vggt_attn_shape* shape, const void* qkv,
+                    const float* q_gamma, const float* q_beta,
+                    const float* k_gamma, const float* k_beta, void* out,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Global mode: all S*T tokens form one sequence.  Writes all of `out`. */
+int vggt_attn_global(const vggt_attn_shape* shape, const void* qkv,
+                     const float* q_gamma, const float* q_beta,
+                     const float* k_gamma, const float* k_beta, void* out,
+                     void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Register mode: the n_special tokens of every frame attend over the
+ * S*n_special special tokens.  Writes only rows t < n_special of `out`. */
+int vggt_attn_register(const vggt_attn_shape* shape, const void* qkv,
+                       const float* q_gamma, const float* q_beta,
+                       const float* k_gamma, const float* k_beta, void* out,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* The two stages of the calls above, exposed so a caller can time or
+ * schedule them separately.  vggt_attn_{frame,global,register} == prologue
+ * followed by core on the same stream.
+ *   prologue: QK-LayerNorm + RoPE of q and k (and, in register mode, the
+ *             gather of the special tokens' v) into `workspace`; also clears
+ *             the workspace status word.
+ *   core:     attention over the packed workspace, writing `out`.
+ * `qkv` is read by both stages (core reads v from it in frame/global mode). */
+int vggt_attn_prologue(int mode, const vggt_attn_shape* shape, const void* qkv,
+                       const float* q_gamma, const float* q_beta,
+                       const float* k_gamma, const float* k_beta,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+int vggt_attn_core(int mode, const vggt_attn_shape* shape, const void* qkv, void* out,
+                   void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* Synchronises `cuda_stream`, then reads and clears the status word of
+ * `workspace`.  *status receives 0 or a negative VGGT_ATTN_ERR_* code
+ * recorded by a kernel since the last prologue on this workspace.
+ * Returns VGGT_ATTN_OK or VGGT_ATTN_ERR_CUDA / _INVALID_ARG. */
+int vggt_attn_read_status(void* workspace, void* cuda_stream, int* status);
+
+/* Fault-path self-test: launches one kernel whose bounded wait on an
+ * mbarrier that nothing arrives at runs out after `timeout_us` microseconds
+ * (1..1000000); it records VGGT_ATTN_ERR_TIMEOUT in the status word of
+ * `workspace` (>= 256 bytes) and exits normally.  Used to test the error path
+ * without faulting the GPU. */
+int vggt_attn_selftest_timeout(void* workspace, unsigned timeout_us, void* cuda_stream);
+
+/* Static, human-readable text for a return code. */
+const char* vggt_attn_error_string(int code);
+
+/* VGGT_ATTN_ABI_VERSION of the loaded library. */
+int vggt_attn_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* VGGT_ATTN_H */

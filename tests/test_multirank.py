@@ -1,0 +1,58 @@
+"""Host-side logic of the multi-GPU bench path, run as 2 gloo ranks on CPU:
+each rank gets its own independent workload copy (weak scaling, no data
+exchange) and the timed region is the max over ranks."""
+import os
+import socket
+
+import pytest
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    import datetime
+    import sys
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    r, w, lr = bench.dist_env()
+    plan = bench.shard_plan(w, r, 1003)
+    local_ms = 10.0 + 5.0 * rank                     # rank 1 is the slow one
+    bench.barrier()
+    mx = bench.reduce_max(local_ms)
+    results[rank] = (r, w, lr, plan["seed"], plan["problems"], mx)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_gloo_ranks_shard_and_reduce():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
+        res = dict(results)
+    assert sorted(res) == [0, 1]
+    seeds = {res[r][3] for r in res}
+    assert len(seeds) == 2                            # independent inputs per rank
+    for r in res:
+        assert res[r][0] == r and res[r][1] == world and res[r][4] == 1
+        assert res[r][5] == 15.0                      # max over ranks, seen by every rank
+
+
+def test_single_process_defaults():
+    import bench
+    os.environ.pop("RANK", None)
+    os.environ.pop("WORLD_SIZE", None)
+    assert bench.dist_env()[:2] == (0, 1)
+    assert bench.reduce_max(3.5) == 3.5
+    assert bench.shard_plan(1, 0, 1003)["seed"] == 1003

@@ -1,0 +1,98 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded bf16 inputs, element by element on every compared row.
+Tolerance (the benchmark spec): max-abs <= 2e-2 and relative Frobenius <= 5e-3."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+from parity import MAX_ABS_TOL, REL_FRO_TOL, check_mode, rows, run_gpu, to_device
+
+pytestmark = pytest.mark.gpu
+
+
+def shp(S, H, ns, gh, gw, **kw):
+    return W.Shape(S=S, T=ns + gh * gw, H=H, n_special=ns, grid_h=gh, grid_w=gw, **kw)
+
+
+# ------------------------------------------------------------------ small / ragged (full oracle)
+SMALL = [
+    ("global", shp(2, 4, 5, 8, 8)),           # the tiny workload's shape: 138 tokens, 2 tiles, ragged
+    ("frame", shp(3, 3, 17, 7, 13)),          # T = 108: one ragged tile per frame
+    ("frame", shp(2, 2, 17, 10, 30)),         # T = 317: 3 tiles, ragged 61
+    ("frame", shp(2, 2, 0, 16, 16)),          # no special tokens, T = 256 exactly 2 tiles
+    ("global", shp(3, 2, 17, 6, 8)),          # N = 195
+    ("global", shp(4, 2, 3, 16, 16)),         # N = 1036: 9 tiles, ragged 12
+    ("global", shp(5, 1, 4, 0, 1)),           # specials only (T = n_special = 4)
+    ("register", shp(40, 2, 17, 4, 4)),       # 680 special tokens: 6 tiles, ragged 40
+    ("register", shp(3, 2, 5, 2, 3)),         # 15 special tokens: one small tile
+    ("frame", shp(1, 1, 1, 1, 1)),            # T = 2
+]
+
+
+@pytest.mark.parametrize("mode,shape", SMALL, ids=[f"{m}-S{s.S}T{s.T}H{s.H}" for m, s in SMALL])
+def test_small_shapes_full_oracle(mode, shape):
+    x = W.make_random_inputs(shape, 100 + shape.T)
+    check_mode(mode, shape, x)
+
+
+def test_workload0_global_tiny():
+    w = W.workload(0)
+    check_mode("global", w.shape, W.make_inputs(w))
+
+
+def test_nondefault_softmax_scale_and_eps():
+    shape = shp(2, 2, 5, 6, 7, ln_eps=1e-3, softmax_scale=0.2, rope_base=10.0)
+    check_mode("global", shape, W.make_random_inputs(shape, 7))
+
+
+# ------------------------------------------------------------------ exact special cases
+def test_single_key_returns_v_exactly():
+    shape = W.Shape(S=1, T=1, H=3, n_special=1, grid_h=0, grid_w=1)
+    x = W.make_random_inputs(shape, 21)
+    for mode in ("frame", "global", "register"):
+        out = run_gpu(mode, shape, x)
+        v = O.bf16_to_f64(x["qkv"][:, :, 2]).reshape(1, 3, 64)
+        np.testing.assert_array_equal(rows(out, shape, [0]), v)
+
+
+def test_constant_v_gives_constant_output():
+    shape = shp(3, 2, 17, 10, 12)
+    x = W.make_random_inputs(shape, 22)
+    x["qkv"][:, :, 2] = x["qkv"][0, 0, 2]                   # every token's v = one bf16 vector per head
+    out = run_gpu("global", shape, x)
+    want = O.bf16_to_f64(x["qkv"][0, 0, 2])                  # [H, 64]
+    got = out.float().cpu().numpy().reshape(-1, shape.H, 64)
+    assert np.abs(got - want[None]).max() <= 2 ** -7 * np.abs(want).max()
+
+
+# ------------------------------------------------------------------ the workloads at full size (sampled)
+def test_workload1_frame_full():
+    w = W.workload(1)
+    check_mode("frame", w.shape, W.make_inputs(w), count=4096, seed=w.seed)
+
+
+def test_workload2_global_sampled():
+    w = W.workload(2)
+    check_mode("global", w.shape, W.make_inputs(w), count=2048, seed=w.seed)
+
+
+@pytest.mark.slow
+def test_workload3_global_long_sampled():
+    w = W.workload(3)
+    check_mode("global", w.shape, W.make_inputs(w), count=4096, seed=w.seed)
+
+
+@pytest.mark.slow
+def test_workload4_register_then_frame():
+    w = W.workload(4)
+    x = W.make_inputs(w)
+    dev = to_device(x)
+    from parity import assert_close, query_sample
+    out_r = run_gpu("register", w.shape, dev_inputs=dev)
+    q = query_sample("register", w.shape, 1 << 62, w.seed)  # all 8,500 special tokens
+    assert_close(rows(out_r, w.shape, q), O.attn_register(w.shape, x, q), "register S=500")
+    del out_r
+    out_f = run_gpu("frame", w.shape, dev_inputs=dev)
+    q = query_sample("frame", w.shape, 4096, w.seed)
+    assert_close(rows(out_f, w.shape, q), O.attn_frame(w.shape, x, q), "frame S=500")

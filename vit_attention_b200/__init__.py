@@ -1,0 +1,179 @@
+"""Python binding of libvggt_attn.so (argument marshalling only).
+
+Every function here has the name of the C entry point it wraps (see
+include/vggt_attn.h) and only converts arguments: tensors become device
+pointers, the shape becomes the C struct, the stream defaults to torch's
+current stream.  All computation runs in the library's CUDA kernels; there is
+no fallback.  Importing this package fails loudly when the library has not
+been built (``python -m vit_attention_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libvggt_attn.so")
+
+FRAME, GLOBAL, REGISTER = 0, 1, 2
+MODES = {"frame": FRAME, "global": GLOBAL, "register": REGISTER}
+
+OK = 0
+ERR_INVALID_ARG = -1
+ERR_UNSUPPORTED_SHAPE = -2
+ERR_MISALIGNED = -3
+ERR_WORKSPACE_TOO_SMALL = -4
+ERR_CUDA = -5
+ERR_TIMEOUT = -6
+ERR_UNSUPPORTED_DEVICE = -7
+
+
+class vggt_attn_shape(ctypes.Structure):  # noqa: N801 - C name
+    _fields_ = [("S", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int), ("head_dim", ctypes.c_int),
+                ("n_special", ctypes.c_int), ("grid_h", ctypes.c_int), ("grid_w", ctypes.c_int),
+                ("ln_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
+
+
+class VggtAttnError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {code} ({error_string(code)})")
+
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m vit_attention_b200.build` "
+                      "(the CUDA library is required; there is no CPU path)")
+_lib = ctypes.CDLL(LIB_PATH)
+
+_vp, _sz, _int = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int
+_shape_p = ctypes.POINTER(vggt_attn_shape)
+_fp = ctypes.c_void_p  # float* passed as a raw device address
+_MODE_SIG = [_shape_p, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]
+_SIGNATURES = {
+    "vggt_attn_workspace_size": (_sz, [_shape_p, _int]),
+    "vggt_attn_frame": (_int, _MODE_SIG),
+    "vggt_attn_global": (_int, _MODE_SIG),
+    "vggt_attn_register": (_int, _MODE_SIG),
+    "vggt_attn_prologue": (_int, [_int, _shape_p, _vp, _fp, _fp, _fp, _fp, _vp, _sz, _vp]),
+    "vggt_attn_core": (_int, [_int, _shape_p, _vp, _vp, _vp, _sz, _vp]),
+    "vggt_attn_read_status": (_int, [_vp, _vp, ctypes.POINTER(ctypes.c_int)]),
+    "vggt_attn_selftest_timeout": (_int, [_vp, ctypes.c_uint, _vp]),
+    "vggt_attn_error_string": (ctypes.c_char_p, [_int]),
+    "vggt_attn_abi_version": (_int, []),
+}
+for _name, (_res, _args) in _SIGNATURES.items():
+    _f = getattr(_lib, _name)
+    _f.restype, _f.argtypes = _res, _args
+
+
+def library():
+    """The loaded ctypes library (for tests that call the C ABI directly)."""
+    return _lib
+
+
+def make_shape(shape) -> vggt_attn_shape:
+    """C struct from any object with the struct's field names (or the struct itself)."""
+    if isinstance(shape, vggt_attn_shape):
+        return shape
+    return vggt_attn_shape(shape.S, shape.T, shape.H, getattr(shape, "head_dim", 64), shape.n_special,
+                           shape.grid_h, shape.grid_w, getattr(shape, "ln_eps", 1e-5),
+                           getattr(shape, "rope_base", 100.0), getattr(shape, "softmax_scale", 0.0))
+
+
+def _ptr(x) -> int:
+    if x is None:
+        return 0
+    if isinstance(x, int):
+        return x
+    return x.data_ptr()
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _nbytes(ws, workspace_bytes):
+    if workspace_bytes is not None:
+        return workspace_bytes
+    return ws.numel() * ws.element_size()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != OK:
+        raise VggtAttnError(rc, where)
+
+
+def error_string(code: int) -> str:
+    return _lib.vggt_attn_error_string(code).decode()
+
+
+def vggt_attn_abi_version() -> int:
+    return _lib.vggt_attn_abi_version()
+
+
+def vggt_attn_workspace_size(shape, mode) -> int:
+    mode = MODES.get(mode, mode)
+    return _lib.vggt_attn_workspace_size(ctypes.byref(make_shape(shape)), mode)
+
+
+def _mode_call(fn, name, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes, stream):
+    s = make_shape(shape)
+    rc = fn(ctypes.byref(s), _ptr(qkv), _ptr(q_gamma), _ptr(q_beta), _ptr(k_gamma), _ptr(k_beta), _ptr(out),
+            _ptr(workspace), _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, name)
+
+
+def vggt_attn_frame(shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes=None, stream=None):
+    _mode_call(_lib.vggt_attn_frame, "vggt_attn_frame", shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out,
+               workspace, workspace_bytes, stream)
+
+
+def vggt_attn_global(shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes=None, stream=None):
+    _mode_call(_lib.vggt_attn_global, "vggt_attn_global", shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out,
+               workspace, workspace_bytes, stream)
+
+
+def vggt_attn_register(shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes=None,
+                       stream=None):
+    _mode_call(_lib.vggt_attn_register, "vggt_attn_register", shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out,
+               workspace, workspace_bytes, stream)
+
+
+def vggt_attn_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace, workspace_bytes=None,
+                       stream=None):
+    mode = MODES.get(mode, mode)
+    rc = _lib.vggt_attn_prologue(mode, ctypes.byref(make_shape(shape)), _ptr(qkv), _ptr(q_gamma), _ptr(q_beta),
+                                 _ptr(k_gamma), _ptr(k_beta), _ptr(workspace), _nbytes(workspace, workspace_bytes),
+                                 _stream(stream))
+    _check(rc, "vggt_attn_prologue")
+
+
+def vggt_attn_core(mode, shape, qkv, out, workspace, workspace_bytes=None, stream=None):
+    mode = MODES.get(mode, mode)
+    rc = _lib.vggt_attn_core(mode, ctypes.byref(make_shape(shape)), _ptr(qkv), _ptr(out), _ptr(workspace),
+                             _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_core")
+
+
+def vggt_attn_read_status(workspace, stream=None) -> int:
+    st = ctypes.c_int(0)
+    _check(_lib.vggt_attn_read_status(_ptr(workspace), _stream(stream), ctypes.byref(st)), "vggt_attn_read_status")
+    return st.value
+
+
+def vggt_attn_selftest_timeout(workspace, timeout_us: int, stream=None) -> None:
+    _check(_lib.vggt_attn_selftest_timeout(_ptr(workspace), timeout_us, _stream(stream)),
+           "vggt_attn_selftest_timeout")
+
+
+_ENTRY = {"frame": vggt_attn_frame, "global": vggt_attn_global, "register": vggt_attn_register}
+
+
+def attend(mode: str, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, stream=None):
+    """Dispatch by mode name to vggt_attn_{frame,global,register}."""
+    _ENTRY[mode](shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, None, stream)

@@ -1,0 +1,356 @@
+// Host side of libvggt_attn.so: argument validation, workspace layout, TMA
+// tensor maps and the kernel launches behind the C ABI in vggt_attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attention_sm100.cuh"
+#include "prologue.cuh"
+#include "vggt_attn.h"
+
+namespace {
+
+using vggt::kStatusBytes;
+
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;  // 2 s per wait; no wait in a healthy run is near it
+constexpr int kMaxRopePositions = 3000;                           // grid_h + grid_w (cos/sin table in shared memory)
+
+struct ModeGeometry {
+  long long B;      // independent problems
+  long long L;      // tokens per problem
+  long long n_tok;  // tokens the prologue handles
+  int n_c;          // head rows per token the prologue handles (q, k[, v])
+};
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool valid_mode(int mode) { return mode == VGGT_ATTN_FRAME || mode == VGGT_ATTN_GLOBAL || mode == VGGT_ATTN_REGISTER; }
+
+int check_shape(const vggt_attn_shape* s, int mode) {
+  if (!s || !valid_mode(mode)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(s->ln_eps) || !std::isfinite(s->rope_base) || !std::isfinite(s->softmax_scale))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!(s->ln_eps > 0.f) || !(s->rope_base > 0.f)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (s->head_dim != 64) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (s->S < 1 || s->T < 1 || s->H < 1 || s->n_special < 0 || s->n_special > s->T || s->grid_h < 0 ||
+      s->grid_w < 0)
+    return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (static_cast<long long>(s->n_special) + static_cast<long long>(s->grid_h) * s->grid_w != s->T)
+    return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (s->T > s->n_special && s->grid_w < 1) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (s->grid_h + static_cast<long long>(s->grid_w) > kMaxRopePositions) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (mode == VGGT_ATTN_REGISTER && s->n_special < 1) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (s->H > 65535) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // grid.y
+  const long long n = static_cast<long long>(s->S) * s->T;
+  if (n > (1LL << 31) - 1 - 256) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // int token indices in the core
+  if (mode == VGGT_ATTN_FRAME && s->S > 65535) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // grid.z
+  return VGGT_ATTN_OK;
+}
+
+ModeGeometry geometry(const vggt_attn_shape* s, int mode) {
+  ModeGeometry g;
+  const long long n = static_cast<long long>(s->S) * s->T;
+  switch (mode) {
+    case VGGT_ATTN_FRAME: g = {s->S, s->T, n, 2}; break;
+    case VGGT_ATTN_GLOBAL: g = {1, n, n, 2}; break;
+    default: g = {1, static_cast<long long>(s->S) * s->n_special, static_cast<long long>(s->S) * s->n_special, 3};
+  }
+  return g;
+}
+
+struct WorkspaceView {
+  int* status;
+  uint16_t* q;
+  uint16_t* k;
+  uint16_t* v;  // register mode only
+  size_t bytes;
+};
+
+WorkspaceView workspace_view(const vggt_attn_shape* s, int mode, void* ws) {
+  const ModeGeometry g = geometry(s, mode);
+  const size_t qk_bytes = align256(static_cast<size_t>(g.B * g.L) * s->H * 64 * 2);
+  WorkspaceView w;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  w.status = reinterpret_cast<int*>(base);
+  w.q = reinterpret_cast<uint16_t*>(base + kStatusBytes);
+  w.k = reinterpret_cast<uint16_t*>(base + kStatusBytes + qk_bytes);
+  size_t total = kStatusBytes + 2 * qk_bytes;
+  w.v = nullptr;
+  if (mode == VGGT_ATTN_REGISTER) {
+    w.v = reinterpret_cast<uint16_t*>(base + total);
+    total += align256(static_cast<size_t>(g.L) * s->H * 64 * 2);
+  }
+  w.bytes = total;
+  return w;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  if (major != 10 || minor != 0) return VGGT_ATTN_ERR_UNSUPPORTED_DEVICE;
+  return VGGT_ATTN_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  });
+  return fn;
+}
+
+// bf16 tensor map, 128-byte swizzle, box inner dim 64 (= 128 B), zero fill out of bounds.
+bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* dims, const cuuint64_t* strides_bytes,
+              const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides_bytes, box,
+            elem_strides, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const float* gq, const float* bq,
+                    const float* gk, const float* bk, const WorkspaceView& w, cudaStream_t stream) {
+  const ModeGeometry g = geometry(s, mode);
+  vggt::PrologueParams p;
+  p.qkv = static_cast<const uint16_t*>(qkv);
+  p.gamma[0] = gq;
+  p.gamma[1] = gk;
+  p.beta[0] = bq;
+  p.beta[1] = bk;
+  p.ws_qk[0] = w.q;
+  p.ws_qk[1] = w.k;
+  p.ws_v = w.v;
+  p.status = w.status;
+  p.n_rows = g.n_tok * g.n_c * s->H;
+  p.S = s->S;
+  p.T = s->T;
+  p.H = s->H;
+  p.n_special = s->n_special;
+  p.grid_h = s->grid_h;
+  p.grid_w = s->grid_w;
+  p.mode = mode;
+  p.L = static_cast<int>(g.L);
+  p.n_c = g.n_c;
+  p.eps = s->ln_eps;
+  const double scale = s->softmax_scale > 0.f ? static_cast<double>(s->softmax_scale) : 1.0 / std::sqrt(64.0);
+  p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
+  p.rope_base = s->rope_base;
+
+  const int threads = 256;
+  const long long groups = p.n_rows;
+  long long blocks = (groups * 8 + threads - 1) / threads;
+  const long long cap = 148LL * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  const size_t smem = static_cast<size_t>(s->grid_h + s->grid_w) * 16 * sizeof(float2);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(vggt::qk_norm_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  vggt::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, const WorkspaceView& w,
+                cudaStream_t stream) {
+  const ModeGeometry g = geometry(s, mode);
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(g.L), static_cast<cuuint64_t>(g.B * s->H)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(g.L) * 128};
+    const cuuint32_t box[3] = {64, 128, 1};
+    if (!make_map(&mq, w.q, 3, dims, strides, box) || !make_map(&mk, w.k, 3, dims, strides, box))
+      return VGGT_ATTN_ERR_CUDA;
+  }
+  {
+    const cuuint32_t box[4] = {64, 1, 128, 1};
+    if (mode == VGGT_ATTN_REGISTER) {  // gathered v: [L][H][64]
+      const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(s->H), static_cast<cuuint64_t>(g.L), 1};
+      const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(s->H) * 128,
+                                     static_cast<cuuint64_t>(g.L) * s->H * 128};
+      if (!make_map(&mv, w.v, 4, dims, strides, box)) return VGGT_ATTN_ERR_CUDA;
+    } else {  // v straight from qkv[S][T][3][H][64]: (dim, head, token, problem)
+      const cuuint64_t tok = static_cast<cuuint64_t>(3) * s->H * 128;
+      const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(s->H), static_cast<cuuint64_t>(g.L),
+                                  static_cast<cuuint64_t>(g.B)};
+      const cuuint64_t strides[3] = {128, tok, tok * static_cast<cuuint64_t>(g.L)};
+      const uint8_t* vbase = static_cast<const uint8_t*>(qkv) + static_cast<size_t>(2) * s->H * 128;
+      if (!make_map(&mv, vbase, 4, dims, strides, box)) return VGGT_ATTN_ERR_CUDA;
+    }
+  }
+  vggt::CoreParams p;
+  p.L = static_cast<int>(g.L);
+  p.H = s->H;
+  p.out_T = s->T;
+  p.out_group = mode == VGGT_ATTN_REGISTER ? s->n_special : static_cast<int>(g.L);
+  p.out = static_cast<uint16_t*>(out);
+  p.status = w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  if (cudaFuncSetAttribute(vggt::attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           vggt::core::SMEM_ALLOC) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>((g.L + vggt::core::BM - 1) / vggt::core::BM), static_cast<unsigned>(s->H),
+                  static_cast<unsigned>(g.B));
+  vggt::attn_core_kernel<<<grid, vggt::core::THREADS, vggt::core::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+  return x < y + nb && y < x + na;
+}
+
+int check_common(int mode, const vggt_attn_shape* s, const void* qkv, void* ws, size_t ws_bytes) {
+  int rc = check_shape(s, mode);
+  if (rc) return rc;
+  if (!qkv || !ws) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(qkv, 16) || !aligned(ws, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  if (ws_bytes < vggt_attn_workspace_size(s, mode)) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  return VGGT_ATTN_OK;
+}
+
+int check_prologue_args(int mode, const vggt_attn_shape* s, const void* qkv, const float* gq, const float* bq,
+                        const float* gk, const float* bk, void* ws, size_t ws_bytes) {
+  int rc = check_common(mode, s, qkv, ws, ws_bytes);
+  if (rc) return rc;
+  if (!gq || !bq || !gk || !bk) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(gq, 16) || !aligned(bq, 16) || !aligned(gk, 16) || !aligned(bk, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t qkv_bytes = static_cast<size_t>(s->S) * s->T * 3 * s->H * 64 * 2;
+  if (overlaps(ws, ws_bytes, qkv, qkv_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+int check_core_args(int mode, const vggt_attn_shape* s, const void* qkv, void* out, void* ws, size_t ws_bytes) {
+  int rc = check_common(mode, s, qkv, ws, ws_bytes);
+  if (rc) return rc;
+  if (!out) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t qkv_bytes = static_cast<size_t>(s->S) * s->T * 3 * s->H * 64 * 2;
+  const size_t out_bytes = static_cast<size_t>(s->S) * s->T * s->H * 64 * 2;
+  if (overlaps(out, out_bytes, qkv, qkv_bytes) || overlaps(out, out_bytes, ws, ws_bytes))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+int run_mode(int mode, const vggt_attn_shape* s, const void* qkv, const float* gq, const float* bq, const float* gk,
+             const float* bk, void* out, void* ws, size_t ws_bytes, void* stream) {
+  int rc = check_prologue_args(mode, s, qkv, gq, bq, gk, bk, ws, ws_bytes);
+  if (rc) return rc;
+  rc = check_core_args(mode, s, qkv, out, ws, ws_bytes);
+  if (rc) return rc;
+  if ((rc = check_device())) return rc;
+  const WorkspaceView w = workspace_view(s, mode, ws);
+  rc = launch_prologue(mode, s, qkv, gq, bq, gk, bk, w, static_cast<cudaStream_t>(stream));
+  if (rc) return rc;
+  return launch_core(mode, s, qkv, out, w, static_cast<cudaStream_t>(stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t vggt_attn_workspace_size(const vggt_attn_shape* shape, int mode) {
+  if (check_shape(shape, mode) != VGGT_ATTN_OK) return 0;
+  return workspace_view(shape, mode, nullptr).bytes;
+}
+
+int vggt_attn_frame(const vggt_attn_shape* shape, const void* qkv, const float* q_gamma, const float* q_beta,
+                    const float* k_gamma, const float* k_beta, void* out, void* workspace, size_t workspace_bytes,
+                    void* cuda_stream) {
+  return run_mode(VGGT_ATTN_FRAME, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes,
+                  cuda_stream);
+}
+
+int vggt_attn_global(const vggt_attn_shape* shape, const void* qkv, const float* q_gamma, const float* q_beta,
+                     const float* k_gamma, const float* k_beta, void* out, void* workspace, size_t workspace_bytes,
+                     void* cuda_stream) {
+  return run_mode(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes,
+                  cuda_stream);
+}
+
+int vggt_attn_register(const vggt_attn_shape* shape, const void* qkv, const float* q_gamma, const float* q_beta,
+                       const float* k_gamma, const float* k_beta, void* out, void* workspace, size_t workspace_bytes,
+                       void* cuda_stream) {
+  return run_mode(VGGT_ATTN_REGISTER, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace,
+                  workspace_bytes, cuda_stream);
+}
+
+int vggt_attn_prologue(int mode, const vggt_attn_shape* shape, const void* qkv, const float* q_gamma,
+                       const float* q_beta, const float* k_gamma, const float* k_beta, void* workspace,
+                       size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_prologue_args(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace, workspace_bytes);
+  if (rc) return rc;
+  if ((rc = check_device())) return rc;
+  return launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace_view(shape, mode, workspace),
+                         static_cast<cudaStream_t>(cuda_stream));
+}
+
+int vggt_attn_core(int mode, const vggt_attn_shape* shape, const void* qkv, void* out, void* workspace,
+                   size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_core_args(mode, shape, qkv, out, workspace, workspace_bytes);
+  if (rc) return rc;
+  if ((rc = check_device())) return rc;
+  return launch_core(mode, shape, qkv, out, workspace_view(shape, mode, workspace),
+                     static_cast<cudaStream_t>(cuda_stream));
+}
+
+int vggt_attn_read_status(void* workspace, void* cuda_stream, int* status) {
+  if (!workspace || !status) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  vggt::StatusBlock host{0, 0};
+  if (cudaMemcpyAsync(&host, workspace, sizeof(host), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  if (cudaMemsetAsync(workspace, 0, sizeof(host), st) != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  *status = host.code;
+  return VGGT_ATTN_OK;
+}
+
+int vggt_attn_selftest_timeout(void* workspace, unsigned timeout_us, void* cuda_stream) {
+  if (!workspace) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  if (timeout_us < 1 || timeout_us > 1000000) return VGGT_ATTN_ERR_INVALID_ARG;
+  int rc = check_device();
+  if (rc) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (cudaMemsetAsync(workspace, 0, sizeof(vggt::StatusBlock), st) != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  vggt::selftest_timeout_kernel<<<1, 32, 0, st>>>(static_cast<int*>(workspace), 1000ull * timeout_us);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+const char* vggt_attn_error_string(int code) {
+  switch (code) {
+    case VGGT_ATTN_OK: return "ok";
+    case VGGT_ATTN_ERR_INVALID_ARG: return "invalid argument (null pointer, bad mode, overlapping buffers or bad scalar)";
+    case VGGT_ATTN_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (head_dim must be 64, T == n_special + grid_h*grid_w, sizes in range)";
+    case VGGT_ATTN_ERR_MISALIGNED: return "misaligned pointer (qkv/out/gamma/beta need 16 bytes, workspace 256 bytes)";
+    case VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL: return "workspace smaller than vggt_attn_workspace_size()";
+    case VGGT_ATTN_ERR_CUDA: return "CUDA runtime, driver or launch error";
+    case VGGT_ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
+    case VGGT_ATTN_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    default: return "unknown error code";
+  }
+}
+
+int vggt_attn_abi_version(void) { return VGGT_ATTN_ABI_VERSION; }
+
+}  // extern "C"

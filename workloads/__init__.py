@@ -24,14 +24,16 @@ Value recipe (no dataset is used; the shapes stand in for the pages'
     describes, "04 method").
   * gamma = 1 + 0.1 N(0,1), beta = 0.1 N(0,1), separately for q and k.
 
-Seeds: qkv uses ``default_rng(seed)``; the affine parameters use
+Seeds: frame ``s`` of qkv uses ``default_rng([seed, 0, s])``; the affine parameters use
 ``default_rng([seed, 1])``; query subsets use ``default_rng([seed, 2])``; the
 shared low-rank component uses ``default_rng([seed, 3])``.  The seed of
 workload ``i`` in ``WORKLOADS`` is ``1000 + i``.
 """
 from __future__ import annotations
 
+import concurrent.futures
 import dataclasses
+import os
 from typing import Dict, List, Optional
 
 import numpy as np
@@ -122,21 +124,29 @@ def make_norm_params(H: int, seed: int, head_dim: int = HEAD_DIM) -> Dict[str, n
 def make_qkv(shape: Shape, seed: int, lowrank: float = 0.0) -> np.ndarray:
     """Seeded bf16 ``qkv[S, T, 3, H, head_dim]`` bit patterns (uint16).
 
-    Drawn frame by frame from one generator so the result does not depend on
-    how much memory is available.
+    Frame ``s`` is drawn from its own generator ``default_rng([seed, 0, s])``,
+    so frames can be drawn in parallel and the result does not depend on the
+    number of threads.
     """
     S, T, H, D = shape.S, shape.T, shape.H, shape.head_dim
-    rng = np.random.default_rng(seed)
     shared = None
     if lowrank:
         shared = (lowrank * np.random.default_rng([seed, 3]).standard_normal(
             (T, 3, H, D), dtype=np.float32)).astype(np.float32)
     bits = np.empty((S, T, 3, H, D), dtype=np.uint16)
-    for s in range(S):
-        z = rng.standard_normal((T, 3, H, D), dtype=np.float32)
+
+    def draw(s: int) -> None:
+        z = np.random.default_rng([seed, 0, s]).standard_normal((T, 3, H, D), dtype=np.float32)
         if shared is not None:
             z += shared
         bits[s] = f32_to_bf16_bits(z)
+
+    if S * T * 3 * H * D >= (1 << 22):
+        with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
+            list(ex.map(draw, range(S)))
+    else:
+        for s in range(S):
+            draw(s)
     return bits
 
 
