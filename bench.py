@@ -272,7 +272,9 @@ def run_ours(args):
     torch.cuda.set_device(device)
     stream = torch.cuda.current_stream(device)
 
-    w = W.workload(HEADLINE)
+    w = W.workload(args.workload)
+    if w.modes != ("global",):
+        raise SystemExit("--workload must name a global-mode workload")
     shape = w.shape
     plan = shard_plan(world, rank, w.seed)
     x = W.make_random_inputs(shape, plan["seed"], w.lowrank) if rank else W.make_inputs(w)
@@ -377,7 +379,8 @@ def run_ours(args):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "mode": "global", "frames": shape.S, "tokens": shape.S * shape.T,
                        "heads": shape.H, "head_dim": 64, "flops_per_step_per_gpu": flops,
-                       "l2": "no flush: qkv 633 MB + workspace 422 MB per step exceed the 126 MB L2",
+                       "l2": f"no flush: qkv {qkv.numel() * 2 / 1e6:.0f} MB + workspace {ws_bytes / 1e6:.0f} MB read per "
+                             "step exceed the 126 MB L2",
                        "parallelism": f"independent replicas x{world} (weak)"},
             "pct_of_peak": 100.0 * value / world / peak,
             "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
@@ -426,6 +429,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-queries", type=int, default=24, help="oracle sample size of the CPU baseline")
     ap.add_argument("--ref-queries", type=int, default=8, help="oracle queries per step of --impl reference")
+    ap.add_argument("--workload", type=int, default=HEADLINE,
+                    help="index of a global-mode workload (default: the S=100 headline; 2 = S=24 for profiling)")
     ap.add_argument("--no-modes", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()

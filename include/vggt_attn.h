@@ -48,8 +48,8 @@
  * failure (a bounded wait inside a kernel that ran out) is recorded in the
  * workspace status word and read with vggt_attn_read_status().
  *
- * Thread safety: no mutable global state; concurrent calls on different
- * workspaces are safe.
+ * Thread safety: concurrent calls on different workspaces are safe.  The only
+ * mutable global state is the shared scratch of vggt_attn_noalloc (below).
  */
 #ifndef VGGT_ATTN_H
 #define VGGT_ATTN_H
@@ -72,7 +72,8 @@ enum {
   VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL = -4,
   VGGT_ATTN_ERR_CUDA = -5,              /* a CUDA runtime/driver call or a launch failed */
   VGGT_ATTN_ERR_TIMEOUT = -6,           /* a bounded wait inside a kernel expired (vggt_attn_read_status) */
-  VGGT_ATTN_ERR_UNSUPPORTED_DEVICE = -7 /* current device is not compute capability 10.0 (sm_100a) */
+  VGGT_ATTN_ERR_UNSUPPORTED_DEVICE = -7, /* current device is not compute capability 10.0 (sm_100a) */
+  VGGT_ATTN_ERR_SCRATCH_TOO_SMALL = -8   /* vggt_attn_noalloc: the problem needs more than VGGT_ATTN_NOALLOC_SCRATCH_BYTES */
 };
 
 /* Attention modes. */
@@ -146,6 +147,41 @@ const char* vggt_attn_error_string(int code);
 
 /* VGGT_ATTN_ABI_VERSION of the loaded library. */
 int vggt_attn_abi_version(void);
+
+/* ------------------------------------------------------------------------
+ * Allocation-free variant (library addition; the pages have no counterpart).
+ *
+ * Some callers cannot hand the library a workspace: a plug-in interface that
+ * passes only input and output buffers, code that must not call cudaMalloc or
+ * cudaFree (cudaFree synchronises the whole device), or a process whose
+ * device-memory budget is fixed at start-up.  vggt_attn_noalloc runs the same
+ * prologue and attention kernels as vggt_attn_frame / _global / _register
+ * (selected by `mode`), but its workspace is a fixed scratch array inside the
+ * library: VGGT_ATTN_NOALLOC_SCRATCH_BYTES (64 MiB) of device memory that every
+ * GPU which loads the library holds until the process exits.
+ *
+ *   - Nothing is allocated: no cudaMalloc, no cudaFree, no allocating library
+ *     routine.  The caller still owns and passes qkv, gamma/beta and out.
+ *   - Problems whose workspace (vggt_attn_workspace_size) exceeds the scratch
+ *     are rejected with VGGT_ATTN_ERR_SCRATCH_TOO_SMALL before anything runs.
+ *     Global mode fits up to S*T*H ~ 262,000 token-heads (e.g. 15 frames of
+ *     1031 tokens x 16 heads); register mode up to S*n_special*H ~ 174,000.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *     first call before any stream capture on the device.
+ *   - All calls share the one array, and it keeps the last call's contents
+ *     (the prologue clears the status word each call; everything else is fully
+ *     rewritten before it is read).  Calls that may overlap on the GPU -- on
+ *     different streams, or from different threads without ordering -- race
+ *     on it; serialise them.
+ *   - A device-side timeout is recorded in the shared scratch; it is not
+ *     readable through this entry point.
+ * Arguments and errors are otherwise those of vggt_attn_frame. */
+#define VGGT_ATTN_NOALLOC_SCRATCH_BYTES (64u << 20)
+int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const void* qkv,
+                      const float* q_gamma, const float* q_beta,
+                      const float* k_gamma, const float* k_beta, void* out,
+                      void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -26,6 +26,8 @@ ERR_WORKSPACE_TOO_SMALL = -4
 ERR_CUDA = -5
 ERR_TIMEOUT = -6
 ERR_UNSUPPORTED_DEVICE = -7
+ERR_SCRATCH_TOO_SMALL = -8
+NOALLOC_SCRATCH_BYTES = 64 << 20
 
 
 class vggt_attn_shape(ctypes.Structure):  # noqa: N801 - C name
@@ -60,6 +62,7 @@ _SIGNATURES = {
     "vggt_attn_selftest_timeout": (_int, [_vp, ctypes.c_uint, _vp]),
     "vggt_attn_error_string": (ctypes.c_char_p, [_int]),
     "vggt_attn_abi_version": (_int, []),
+    "vggt_attn_noalloc": (_int, [_int, _shape_p, _vp, _fp, _fp, _fp, _fp, _vp, _vp]),
 }
 for _name, (_res, _args) in _SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -169,6 +172,16 @@ def vggt_attn_read_status(workspace, stream=None) -> int:
 def vggt_attn_selftest_timeout(workspace, timeout_us: int, stream=None) -> None:
     _check(_lib.vggt_attn_selftest_timeout(_ptr(workspace), timeout_us, _stream(stream)),
            "vggt_attn_selftest_timeout")
+
+
+def vggt_attn_noalloc(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, stream=None):
+    """Same computation as vggt_attn_{frame,global,register}, for callers that
+    cannot give the library a workspace: the library uses its own fixed
+    64 MiB device scratch instead (shared by all calls; serialise calls)."""
+    mode = MODES.get(mode, mode)
+    rc = _lib.vggt_attn_noalloc(mode, ctypes.byref(make_shape(shape)), _ptr(qkv), _ptr(q_gamma), _ptr(q_beta),
+                                _ptr(k_gamma), _ptr(k_beta), _ptr(out), _stream(stream))
+    _check(rc, "vggt_attn_noalloc")
 
 
 _ENTRY = {"frame": vggt_attn_frame, "global": vggt_attn_global, "register": vggt_attn_register}

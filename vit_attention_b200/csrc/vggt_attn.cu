@@ -347,6 +347,7 @@ const char* vggt_attn_error_string(int code) {
     case VGGT_ATTN_ERR_CUDA: return "CUDA runtime, driver or launch error";
     case VGGT_ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
     case VGGT_ATTN_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
+    case VGGT_ATTN_ERR_SCRATCH_TOO_SMALL: return "problem needs more workspace than the fixed 64 MiB scratch of vggt_attn_noalloc";
     default: return "unknown error code";
   }
 }
@@ -354,3 +355,50 @@ const char* vggt_attn_error_string(int code) {
 int vggt_attn_abi_version(void) { return VGGT_ATTN_ABI_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.  For callers that cannot allocate device
+// memory (plug-in interfaces that pass only inputs and outputs, code that must
+// not call cudaMalloc/cudaFree, fixed device-memory budgets): the workspace is
+// this file-scope array, which every GPU that loads the library holds until
+// the process exits.  In host code `noalloc_scratch` names a host-side stand-in,
+// not the device memory, so its device address is looked up once per device
+// with cudaGetSymbolAddress and only that address is passed to the kernels.
+namespace {
+
+static __device__ __align__(256) unsigned char noalloc_scratch[VGGT_ATTN_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex noalloc_mutex;
+void* noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the scratch array on the current device (set-up on the
+// first call per device, with that device current).
+int noalloc_scratch_address(void** ptr) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VGGT_ATTN_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(noalloc_mutex);
+  if (!noalloc_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, noalloc_scratch) != cudaSuccess || p == nullptr) return VGGT_ATTN_ERR_CUDA;
+    noalloc_ptr[dev] = p;
+  }
+  *ptr = noalloc_ptr[dev];
+  return VGGT_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const void* qkv, const float* q_gamma,
+                                 const float* q_beta, const float* k_gamma, const float* k_beta, void* out,
+                                 void* cuda_stream) {
+  int rc = check_shape(shape, mode);
+  if (rc) return rc;
+  if (vggt_attn_workspace_size(shape, mode) > VGGT_ATTN_NOALLOC_SCRATCH_BYTES) return VGGT_ATTN_ERR_SCRATCH_TOO_SMALL;
+  if ((rc = check_device())) return rc;
+  void* scratch = nullptr;
+  if ((rc = noalloc_scratch_address(&scratch))) return rc;
+  return run_mode(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, scratch, VGGT_ATTN_NOALLOC_SCRATCH_BYTES,
+                  cuda_stream);
+}
+
