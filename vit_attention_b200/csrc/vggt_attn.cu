@@ -207,7 +207,8 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   if (cudaFuncSetAttribute(vggt::attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            vggt::core::SMEM_ALLOC) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
-  const dim3 grid(static_cast<unsigned>((g.L + vggt::core::BM - 1) / vggt::core::BM), static_cast<unsigned>(s->H),
+  constexpr int rows_per_cta = vggt::core::BM * vggt::core::NQ;
+  const dim3 grid(static_cast<unsigned>((g.L + rows_per_cta - 1) / rows_per_cta), static_cast<unsigned>(s->H),
                   static_cast<unsigned>(g.B));
   vggt::attn_core_kernel<<<grid, vggt::core::THREADS, vggt::core::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
