@@ -207,6 +207,14 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   if (cudaFuncSetAttribute(vggt::attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            vggt::core::SMEM_ALLOC) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
+  // The kernel re-splits its registers between warpgroups (setmaxnreg); that
+  // split assumes the compiled per-thread count.  A build with fewer registers
+  // at launch would make the softmax warps wait forever for registers, so
+  // refuse to launch it.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, vggt::attn_core_kernel) != cudaSuccess ||
+      fa.numRegs < vggt::core::REGS_AT_LAUNCH)
+    return VGGT_ATTN_ERR_CUDA;
   constexpr int rows_per_cta = vggt::core::BM * vggt::core::NQ;
   const dim3 grid(static_cast<unsigned>((g.L + rows_per_cta - 1) / rows_per_cta), static_cast<unsigned>(s->H),
                   static_cast<unsigned>(g.B));
