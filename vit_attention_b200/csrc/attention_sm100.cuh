@@ -54,6 +54,7 @@ namespace vggt {
 struct CoreParams {
   int L;              // keys (and queries) per problem
   int H;              // heads
+  int B;              // problems
   int out_T;          // tokens per frame of `out`
   int out_group;      // query i of problem b -> out row b*out_T + (i/out_group)*out_T + i%out_group
   uint16_t* out;      // bf16 [.][H][64]
@@ -85,6 +86,7 @@ constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;          // slack to align the base to 1024 B
 constexpr int THREADS = 640;
+constexpr bool PERSISTENT = false;                  // grid: one CTA per SM over all units, or one CTA per unit
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TILE_COLS = 256;                    // TMEM columns per Q tile
 constexpr uint32_t COL_O = 128;                       // O_i0 offset inside a tile's columns (O_i1 at +64)

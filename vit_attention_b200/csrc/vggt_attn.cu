@@ -48,6 +48,7 @@ int check_shape(const vggt_attn_shape* s, int mode) {
   if (s->H > 65535) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // grid.y
   const long long n = static_cast<long long>(s->S) * s->T;
   if (n > (1LL << 31) - 1 - 256) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // int token indices in the core
+  if (n * 3 * s->H > (1LL << 31) - 1) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // int row indices in the prologue
   if (mode == VGGT_ATTN_FRAME && s->S > 65535) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // grid.z
   return VGGT_ATTN_OK;
 }
@@ -154,9 +155,10 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
   p.rope_base = s->rope_base;
 
+  // One block per token (grid-stride over tokens, four at a time), at most
+  // 8 blocks per SM.
   const int threads = 256;
-  const long long groups = p.n_rows;
-  long long blocks = (groups * 8 + threads - 1) / threads;
+  long long blocks = g.n_tok;
   const long long cap = 148LL * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
@@ -176,12 +178,13 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   {
     const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(g.L), static_cast<cuuint64_t>(g.B * s->H)};
     const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(g.L) * 128};
-    const cuuint32_t box[3] = {64, 128, 1};
-    if (!make_map(&mq, w.q, 3, dims, strides, box) || !make_map(&mk, w.k, 3, dims, strides, box))
+    const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};   // one query tile
+    const cuuint32_t box_k[3] = {64, vggt::core::BN, 1};   // one key tile
+    if (!make_map(&mq, w.q, 3, dims, strides, box_q) || !make_map(&mk, w.k, 3, dims, strides, box_k))
       return VGGT_ATTN_ERR_CUDA;
   }
   {
-    const cuuint32_t box[4] = {64, 1, 128, 1};
+    const cuuint32_t box[4] = {64, 1, vggt::core::BN, 1};  // one value tile
     if (mode == VGGT_ATTN_REGISTER) {  // gathered v: [L][H][64]
       const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(s->H), static_cast<cuuint64_t>(g.L), 1};
       const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(s->H) * 128,
@@ -199,6 +202,7 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   vggt::CoreParams p;
   p.L = static_cast<int>(g.L);
   p.H = s->H;
+  p.B = static_cast<int>(g.B);
   p.out_T = s->T;
   p.out_group = mode == VGGT_ATTN_REGISTER ? s->n_special : static_cast<int>(g.L);
   p.out = static_cast<uint16_t*>(out);
@@ -215,9 +219,19 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   if (cudaFuncGetAttributes(&fa, vggt::attn_core_kernel) != cudaSuccess ||
       fa.numRegs < vggt::core::REGS_AT_LAUNCH)
     return VGGT_ATTN_ERR_CUDA;
-  constexpr int rows_per_cta = vggt::core::BM * vggt::core::NQ;
-  const dim3 grid(static_cast<unsigned>((g.L + rows_per_cta - 1) / rows_per_cta), static_cast<unsigned>(s->H),
-                  static_cast<unsigned>(g.B));
+  constexpr int rows_per_unit = vggt::core::BM * vggt::core::NQ;
+  const long long n_qp = (g.L + rows_per_unit - 1) / rows_per_unit;
+  dim3 grid(static_cast<unsigned>(n_qp), static_cast<unsigned>(s->H), static_cast<unsigned>(g.B));
+  if (vggt::core::PERSISTENT) {
+    // One CTA per SM walks the work units (query pair x head x problem).
+    const long long n_units = n_qp * s->H * g.B;
+    int dev = 0, n_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
+      return VGGT_ATTN_ERR_CUDA;
+    if (n_units > 0x7FFFFFFFLL) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+    grid = dim3(static_cast<unsigned>(n_units < n_sm ? n_units : n_sm));
+  }
   vggt::attn_core_kernel<<<grid, vggt::core::THREADS, vggt::core::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
