@@ -7,39 +7,45 @@
 // attention of the alternating-attention block; the kernel is the same for
 // the three modes, only the workspace views and the output row map differ.)
 //
-// Warp roles (640 threads, 20 warps):
-//   warp 0       TMA producer: both Q tiles once, then K/V tiles of 128 keys
-//                through a 4-stage shared-memory ring (128-byte swizzle, no
+// Keys are processed in steps of 64.  Every Q tile has two S buffers in
+// TMEM, so the tensor core computes S(j+2) while the softmax works on S(j)
+// and the softmax never waits for a QK^T product it could have had earlier.
+//
+// Warp roles (384 threads, 12 warps):
+//   warp 0       TMA producer: both Q tiles once, then K/V tiles of 64 keys
+//                through an 8-stage shared-memory ring (128-byte swizzle, no
 //                multicast).
 //   warps 1, 2   MMA issuers, one per Q tile (warp 1 also allocates TMEM).
-//                One thread can issue a tcgen05.mma only every ~45-50 cycles
-//                whatever its size, and the N=64 products below need 32, so
-//                the two tiles' streams are issued by two threads:
-//                  S_i = Q_i K_j^T      (M=128, N=128, K=16 x 4, fp32 in TMEM)
-//                  O_ih += P_ih V_jh    (M=128, N=64,  K=16 x 4 per key half h)
-//                in the order PV_i(j-1), S_i(j) (program order of one thread,
-//                so the commit that publishes S_i(j) also proves that PV_i(j-1)
-//                has finished).  Tile 1 starts once tile 0's first softmax is
-//                done, so the two tiles' softmax phases alternate.
+//                One thread can issue a tcgen05.mma only every ~45-50 cycles,
+//                so the two tiles' streams go out from two threads.  Per step
+//                j a tile's stream is
+//                  O_i += P_i(j) [V_j | 1]  (M=128, N=80, K=16 x 4, P from TMEM)
+//                  S_i(j+2) = Q_i K_j+2^T   (M=128, N=64, K=16 x 4, into the S
+//                                            buffer P_i(j) came from)
+//                in program order, so S(j+2) overwrites P(j) only after PV(j).
+//                The B operand of PV is V_j followed by 16 columns of ones
+//                (a constant shared-memory tile), so columns 64-79 of O_i
+//                accumulate the row sums of P on the tensor core and the
+//                softmax threads never add their probabilities up.
 //   warp 3       idle.
-//   warps 4-19   softmax, four warpgroups: (tile 0, keys 0-63 of every key
-//                tile), (tile 0, keys 64-127), (tile 1, keys 0-63), (tile 1,
-//                keys 64-127).  Each warpgroup runs its own online softmax over
-//                its half of the keys -- running reference max m, sum l and
-//                accumulator O_ih of its own -- so the two halves of a row never
-//                synchronise inside the key loop; they are merged once at the
-//                end: m = max(m_0, m_1), O = sum_h 2^(m_h - m) O_ih and
-//                l = sum_h 2^(m_h - m) l_h.  Thread r of a warpgroup owns query
-//                row r (= TMEM lane r).  Per key tile it reads its 64 scores
-//                from TMEM, writes P = 2^(s - m) as bf16 over the first 32 of
-//                its S columns, and rescales O_ih only when m grows by more than
-//                8 (a factor of 256; below that the stale max is kept, which is
-//                exact because O_ih and l_h always share the same m).  A small
-//                share of the exponentials runs on the FMA pipe (a cubic for
-//                2^f after an exponent split), the rest on the MUFU unit.
-
-// TMEM (512 columns): tile i owns columns 256 i .. 256 i + 255: S/P at +0,
-// O_i0 at +128, O_i1 at +192.  Every mbarrier wait is bounded
+//   warps 4-11   softmax, one warpgroup per Q tile; thread r owns query row r
+//                (= TMEM lane r).  Per step it reads its 64 scores, keeps a
+//                running reference max m in fp32, writes P = 2^(s - m) as
+//                bf16 over the first 32 columns of the S buffer, and rescales
+//                O (head dims and the sum column) in TMEM only when m grows by
+//                more than 8 (a factor of 256; below that the stale max is
+//                kept, which is exact because O and its sum column always
+//                share the same m).  A rescale first waits for the previous PV
+//                to complete.  A small share of the exponentials runs on the
+//                FMA pipe (a cubic for 2^f after an exponent split), the rest
+//                on the MUFU unit.
+//                Epilogue: O[:, 0:64] / O[:, 64] -> bf16 -> out.
+//
+// The row sum is that of the bf16-rounded P that multiplies V, so numerator
+// and denominator see the same rounding.
+//
+// TMEM (512 columns allocated): S buffers of tile i at columns 128 i and
+// 128 i + 64, O_i at 256 + 80 i (80 columns).  Every mbarrier wait is bounded
 // (wait_bounded); on expiry the CTA records VGGT_ATTN_ERR_TIMEOUT in the
 // workspace status word, drains what it has in flight and exits without
 // writing its output tiles.
@@ -63,55 +69,50 @@ struct CoreParams {
 };
 
 namespace core {
-constexpr int BM = 128, BN = 128, D = 64, STAGES = 4, NQ = 2;
-constexpr int HALF = BN / 2;                           // key columns per softmax warpgroup
-constexpr int TILE_BYTES = BM * D * 2;                 // 16 KB (Q, K or V tile)
+constexpr int BM = 128, BN = 64, D = 64, STAGES = 8, NQ = 2;
+constexpr int Q_BYTES = BM * D * 2;                    // 16 KB query tile
+constexpr int KV_BYTES = BN * D * 2;                   // 8 KB key or value tile
 constexpr int OFF_Q = 0;                               // NQ tiles
-constexpr int OFF_K = OFF_Q + NQ * TILE_BYTES;
-constexpr int OFF_V = OFF_K + STAGES * TILE_BYTES;
-constexpr int OFF_XCHG = OFF_V + STAGES * TILE_BYTES;  // float2 [NQ][2 halves][BM]: final (m, l) of each half
-constexpr int OFF_BAR = OFF_XCHG + NQ * 2 * BM * 8;
+constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
+constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+constexpr int OFF_ONES = OFF_V + STAGES * KV_BYTES;    // 64 x 64 bf16 ones: the PV product's extra columns
+constexpr int OFF_BAR = OFF_ONES + KV_BYTES;
 enum {
   BAR_Q = 0,
   BAR_KV_FULL = 1,
   BAR_KV_EMPTY = BAR_KV_FULL + STAGES,
-  BAR_S_FULL = BAR_KV_EMPTY + STAGES,
-  BAR_P_FULL = BAR_S_FULL + NQ,
-  BAR_O_FINAL = BAR_P_FULL + NQ,
-  BAR_XCHG = BAR_O_FINAL + NQ,        // one per (tile, lane quarter): the two halves' warps
-  BAR_DRAIN = BAR_XCHG + NQ * 4,     // one per MMA issuer
+  BAR_S_FULL = BAR_KV_EMPTY + STAGES,   // [tile][buffer]
+  BAR_P_FULL = BAR_S_FULL + NQ * 2,     // [tile][buffer]
+  BAR_PV_DONE = BAR_P_FULL + NQ * 2,    // [tile]
+  BAR_O_FINAL = BAR_PV_DONE + NQ,       // [tile]
+  BAR_DRAIN = BAR_O_FINAL + NQ,         // [issuer]
   N_BARS = BAR_DRAIN + NQ
 };
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;          // slack to align the base to 1024 B
-constexpr int THREADS = 640;
-constexpr bool PERSISTENT = false;                  // grid: one CTA per SM over all units, or one CTA per unit
+constexpr int THREADS = 384;
+constexpr bool PERSISTENT = false;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TILE_COLS = 256;                    // TMEM columns per Q tile
-constexpr uint32_t COL_O = 128;                       // O_i0 offset inside a tile's columns (O_i1 at +64)
+constexpr uint32_t COL_O = 256;                       // O_i (80 columns) at 256 + 80 i
 constexpr float RESCALE_THRESHOLD = 8.0f;              // log2 units
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
-constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);  // V is MN-major (head dim contiguous)
-// Exponentials of score pair q (0..31 in a half row) run on the FMA pipe when
-// bit (q % 8) of this mask is set, on the MUFU unit otherwise.
+// PV has N = 80: the 64 head dims of V, then 16 columns of ones whose
+// products are the row sums of P (every one of columns 64-79 holds it).
+constexpr int NV = D + 16;
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, NV, 0, 1);  // V is MN-major (head dim contiguous)
+// Exponentials of score pair q (0..31 in a row of a step) run on the FMA pipe
+// when bit (q % 8) of this mask is set, on the MUFU unit otherwise.
 constexpr uint32_t POLY_PAIR_MASK = 0x80u;
-// Register split (setmaxnreg): the block launches with REGS_AT_LAUNCH per
-// thread; warpgroup 0 (TMA + MMA warps) gives registers back, the four softmax
-// warpgroups take them.  The sum never exceeds the launch allocation
+// Register split (setmaxnreg): warpgroup 0 gives registers back, the two
+// softmax warpgroups take them; the sum never exceeds the launch allocation
 // (launch_core checks the compiled register count before every launch).
-constexpr int REGS_AT_LAUNCH = 96;
-constexpr int REGS_PRODUCER = 32;
-constexpr int REGS_SOFTMAX = 112;
-static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 512 <= REGS_AT_LAUNCH * THREADS, "register split too large");
+constexpr int REGS_AT_LAUNCH = 168;
+constexpr int REGS_PRODUCER = 56;
+constexpr int REGS_SOFTMAX = 224;
+static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 256 <= REGS_AT_LAUNCH * THREADS, "register split too large");
 }  // namespace core
 
-// 2^x for x <= ~128 on the FMA pipe, two values at once: x = j + f with
-// j = round(x) (via the 1.5*2^23 shift), f in [-1/2, 1/2]; 2^f from a cubic
-// fitted by minimax in relative error (fit_exp2_poly.py, max rel. error
-// 7.5e-5); 2^j added to the exponent field.  x is clamped at -125 so that the
-// exponent field never underflows (2^-125 is far below any probability that
-// survives bf16 rounding next to the row maximum's 1).
 struct PolyConsts {
   uint64_t shift2, c3, c2, c1, c0;   // each: the same fp32 constant in both halves
 };
@@ -123,6 +124,12 @@ __device__ __forceinline__ PolyConsts poly_consts() {
   return {dup_f32(12582912.0f), dup_f32(5.517166853e-02f), dup_f32(2.426111251e-01f), dup_f32(6.932609677e-01f),
           dup_f32(9.999280572e-01f)};
 }
+// 2^x for x <= ~128 on the FMA pipe, two values at once: x = j + f with
+// j = round(x) (via the 1.5*2^23 shift), f in [-1/2, 1/2]; 2^f from a cubic
+// fitted by minimax in relative error (fit_exp2_poly.py, max rel. error
+// 7.5e-5); 2^j added to the exponent field.  x is clamped at -125 so that the
+// exponent field never underflows (2^-125 is far below any probability that
+// survives bf16 rounding next to the row maximum's 1).
 __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1, const PolyConsts& k) {
   x0 = fmaxf(x0, -125.0f);
   x1 = fmaxf(x1, -125.0f);
@@ -139,6 +146,8 @@ __device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, floa
       "mov.b64 {%2, %3}, rp;\n\t}"
       : "=f"(t0), "=f"(t1), "=f"(p0), "=f"(p1)
       : "f"(x0), "f"(x1), "l"(k.shift2), "l"(k.c3), "l"(k.c2), "l"(k.c1), "l"(k.c0));
+  // bits(2^f) + round(x) << 23; the low mantissa bits of t hold round(x) and
+  // the multiply by 2^23 drops the rest of t's bits out of the word.
   uint32_t b0, b1;
   asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(b0) : "r"(__float_as_uint(t0)), "r"(__float_as_uint(p0)));
   asm("mad.lo.u32 %0, %1, 8388608, %2;" : "=r"(b1) : "r"(__float_as_uint(t1)), "r"(__float_as_uint(p1)));
@@ -161,6 +170,14 @@ __device__ __forceinline__ void add_x2(float a0, float a1, float b0, float b1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// 32 lanes x 1 column load / store.
+__device__ __forceinline__ void tmem_ld1(uint32_t taddr, uint32_t& r) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr) : "memory");
+}
+__device__ __forceinline__ void tmem_st1(uint32_t taddr, uint32_t r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x1.b32 [%0], {%1};" ::"r"(taddr), "r"(r) : "memory");
+}
+
 // 32 lanes x 16 columns store.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
   asm volatile(
@@ -171,26 +188,26 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
-// Softmax role of one warp: `tile` (Q tile), `half` (key columns 64*half ..
-// 64*half+63 of every key tile), `quarter` (TMEM lanes / rows 32*quarter ..).
-__device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem, uint32_t bar0, float2* xchg,
+// Softmax warpgroup role: warps 4-7 own Q tile 0, warps 8-11 Q tile 1.
+__device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem, uint32_t bar0,
                                              volatile int* abort_flag, int h, int b, int q0, int n_kv, int warp,
                                              int lane) {
   using namespace core;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
-  const int g = (warp >> 2) - 1;             // softmax warpgroup 0..3
-  const int tile = g >> 1, half = g & 1;
+  const int tile = (warp >> 2) - 1;
   const int quarter = warp & 3;              // TMEM lane quarter this warp may access
   const int row = quarter * 32 + lane;       // query row of this thread in its tile
   const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-  const uint32_t t_base = tmem + lane_base + tile * TILE_COLS;
-  const uint32_t s_addr = t_base + half * HALF;
-  const uint32_t o_addr = t_base + COL_O + half * D;
-  float m_run = -INFINITY, l_run = 0.f;
+  const uint32_t s_base = tmem + lane_base + tile * 2 * BN;
+  const uint32_t o_addr = tmem + lane_base + COL_O + tile * NV;
   const PolyConsts pc = poly_consts();
+  float m_run = -INFINITY;
   bool ok = true;
   for (int j = 0; j < n_kv; ++j) {
-    ok = wait_bounded(bar(BAR_S_FULL + tile), j & 1, abort_flag, p.status, p.timeout_ns, 0x300u | tile);
+    const int buf = j & 1;
+    const uint32_t s_addr = s_base + buf * BN;
+    ok = wait_bounded(bar(BAR_S_FULL + tile * 2 + buf), (j >> 1) & 1, abort_flag, p.status, p.timeout_ns,
+                      0x300u | tile);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
     tc_fence_after();
@@ -198,8 +215,8 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
     tmem_ld32(s_addr, sr[0]);
     tmem_ld32(s_addr + 32, sr[1]);
     tmem_wait_ld();
-    const int valid = p.L - j * BN - half * HALF;   // keys of this half tile that exist
-    if (valid < HALF) {                              // last key tile only (uniform branch)
+    const int valid = p.L - j * BN;          // keys of this step that exist (>= BN except on the last)
+    if (valid < BN) {                        // last step only (uniform branch)
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
@@ -213,16 +230,15 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
       mx1 = max3f(mx1, __uint_as_float(sr[1][e]), __uint_as_float(sr[1][e + 1]));
     }
     const float tile_max = fmaxf(mx0, mx1);
-    // Move the reference max on the first tile, or when it grows by more
-    // than the threshold.  A half with no valid key yet keeps m = -inf.
+    // Move the reference max on the first step, or when it grows by more
+    // than the threshold.
     const bool move = (j == 0) || (tile_max > m_run + RESCALE_THRESHOLD);
     float alpha = 1.f;
     if (move) {
-      alpha = (j == 0 || m_run == -INFINITY) ? 0.f : ex2_approx(m_run - tile_max);
+      alpha = (j == 0) ? 0.f : ex2_approx(m_run - tile_max);
       m_run = tile_max;
     }
-    const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-    float acc0 = 0.f, acc1 = 0.f, acc2 = 0.f, acc3 = 0.f;
+    const float neg_m = -m_run;
 #pragma unroll
     for (int c = 0; c < 2; ++c) {
       uint32_t pk[16];
@@ -237,77 +253,67 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
           p0 = ex2_approx(x0);
           p1 = ex2_approx(x1);
         }
-        if (e & 2) {
-          add_x2(acc2, acc3, p0, p1, acc2, acc3);
-        } else {
-          add_x2(acc0, acc1, p0, p1, acc0, acc1);
-        }
         pk[e >> 1] = pack_bf16x2(p0, p1);
       }
-      // P of this half (64 keys -> 32 columns) overwrites the first 32 of the
-      // half's own 64 S columns: the other half's S is never touched.
+      // P (64 keys -> 32 columns) overwrites the first 32 columns of this S buffer.
       tmem_st16(s_addr + c * 16, pk);
     }
-    l_run = l_run * alpha + ((acc0 + acc1) + (acc2 + acc3));
-    // O_ih must be rescaled before PV_ih(j) accumulates into it.  PV(j-1) is
-    // complete: the commit that published S_i(j) came after it.
-    // Warp-uniform: tcgen05.ld/st are warp-collective.
+    // O must be rescaled before PV(j) accumulates into it, and after PV(j-1)
+    // has: PV(j-2) is known complete (S(j) was issued after it and has
+    // completed), so PV_DONE is at most one phase behind.  Warp-uniform:
+    // tcgen05.ld/st are warp-collective.
     if (__any_sync(0xffffffffu, move && j > 0)) {
-      uint32_t orr[2][32];
+      ok = wait_bounded(bar(BAR_PV_DONE + tile), (j - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x310u | tile);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t orr[2][32], osum;
       tmem_ld32(o_addr, orr[0]);
       tmem_ld32(o_addr + 32, orr[1]);
+      tmem_ld1(o_addr + D, osum);
       tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 2; ++c)
 #pragma unroll
         for (int e = 0; e < 32; ++e) orr[c][e] = __float_as_uint(__uint_as_float(orr[c][e]) * alpha);
+      osum = __float_as_uint(__uint_as_float(osum) * alpha);
       tmem_st32(o_addr, orr[0]);
       tmem_st32(o_addr + 32, orr[1]);
+      tmem_st1(o_addr + D, osum);
     }
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(bar(BAR_P_FULL + tile));
+    mbar_arrive(bar(BAR_P_FULL + tile * 2 + buf));
   }
-  // Merge the two halves of every row: both publish (m_h, l_h), then half h
-  // writes output columns 32h .. 32h+31 from both accumulators.
   if (ok) {
-    xchg[(tile * 2 + half) * BM + row] = make_float2(m_run, l_run);
-    const uint32_t xbar = bar(BAR_XCHG + tile * 4 + quarter);
-    mbar_arrive(xbar);
-    ok = wait_bounded(xbar, 0, abort_flag, p.status, p.timeout_ns, 0x350u | tile) &&
-         wait_bounded(bar(BAR_O_FINAL + tile), 0, abort_flag, p.status, p.timeout_ns, 0x320u | tile);
+    ok = wait_bounded(bar(BAR_O_FINAL + tile), 0, abort_flag, p.status, p.timeout_ns, 0x320u | tile);
     ok = __all_sync(0xffffffffu, ok);
   }
   if (ok) {
     tc_fence_after();
-    const float2 ml0 = xchg[(tile * 2 + 0) * BM + row];
-    const float2 ml1 = xchg[(tile * 2 + 1) * BM + row];
-    const float m = fmaxf(ml0.x, ml1.x);
-    const float a0 = (ml0.x == -INFINITY) ? 0.f : ex2_approx(ml0.x - m);
-    const float a1 = (ml1.x == -INFINITY) ? 0.f : ex2_approx(ml1.x - m);
-    const float inv = 1.f / (a0 * ml0.y + a1 * ml1.y);
-    const float w0 = a0 * inv, w1 = a1 * inv;
-    uint32_t o0[32], o1[32];
-    tmem_ld32(t_base + COL_O + half * 32, o0);        // O_i0, columns 32h..
-    tmem_ld32(t_base + COL_O + D + half * 32, o1);    // O_i1, columns 32h..
+    uint32_t orr[2][32], osum;
+    tmem_ld32(o_addr, orr[0]);
+    tmem_ld32(o_addr + 32, orr[1]);
+    tmem_ld1(o_addr + D, osum);
     tmem_wait_ld();
     const int i = q0 + tile * BM + row;
     if (i < p.L) {
+      const float inv = 1.f / __uint_as_float(osum);
       const long long out_row = static_cast<long long>(b) * p.out_T +
                                 static_cast<long long>(i / p.out_group) * p.out_T + (i % p.out_group);
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D + half * (D / 2));
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D);
 #pragma unroll
-      for (int v = 0; v < 4; ++v) {
-        float f[8];
+      for (int c = 0; c < 2; ++c) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          f[e] = __uint_as_float(o0[v * 8 + e]) * w0 + __uint_as_float(o1[v * 8 + e]) * w1;
-        uint4 w;
-        w.x = pack_bf16x2(f[0], f[1]);
-        w.y = pack_bf16x2(f[2], f[3]);
-        w.z = pack_bf16x2(f[4], f[5]);
-        w.w = pack_bf16x2(f[6], f[7]);
-        dst[v] = w;
+        for (int v = 0; v < 4; ++v) {
+          uint4 w;
+          const uint32_t* o = &orr[c][v * 8];
+          w.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          dst[c * 4 + v] = w;
+        }
       }
     }
   }
@@ -324,7 +330,6 @@ __global__ void __launch_bounds__(core::THREADS, 1)
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
-  float2* xchg = reinterpret_cast<float2*>(smem + OFF_XCHG);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, b = blockIdx.z;
@@ -339,18 +344,23 @@ __global__ void __launch_bounds__(core::THREADS, 1)
       mbar_init(bar(BAR_KV_EMPTY + s), n_tiles);   // one commit per MMA issuer
     }
     for (int i = 0; i < NQ; ++i) {
-      mbar_init(bar(BAR_S_FULL + i), 1);
-      mbar_init(bar(BAR_P_FULL + i), 256);
+      for (int buf = 0; buf < 2; ++buf) {
+        mbar_init(bar(BAR_S_FULL + i * 2 + buf), 1);
+        mbar_init(bar(BAR_P_FULL + i * 2 + buf), 128);
+      }
+      mbar_init(bar(BAR_PV_DONE + i), 1);
       mbar_init(bar(BAR_O_FINAL + i), 1);
+      mbar_init(bar(BAR_DRAIN + i), 1);
     }
-    for (int i = 0; i < NQ * 4; ++i) mbar_init(bar(BAR_XCHG + i), 64);
-    for (int i = 0; i < NQ; ++i) mbar_init(bar(BAR_DRAIN + i), 1);
     fence_mbar_init();
     *abort_flag = status_is_set(p.status) ? 1 : 0;  // another CTA already failed: skip the work
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
   }
+  for (int e = threadIdx.x; e < KV_BYTES / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(smem + OFF_ONES)[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 1) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
     tmem_relinquish();
@@ -363,8 +373,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
 
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    if (!skip && (((warp >> 2) - 1) >> 1) < n_tiles)
-      softmax_role(p, tmem, bar0, xchg, abort_flag, h, b, q0, n_kv, warp, lane);
+    if (!skip && ((warp >> 2) - 1) < n_tiles) softmax_role(p, tmem, bar0, abort_flag, h, b, q0, n_kv, warp, lane);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
   }
@@ -373,9 +382,9 @@ __global__ void __launch_bounds__(core::THREADS, 1)
     if (lane == 0 && !skip) {
       int issued[STAGES];
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
-      mbar_arrive_expect_tx(bar(BAR_Q), n_tiles * TILE_BYTES);
+      mbar_arrive_expect_tx(bar(BAR_Q), n_tiles * Q_BYTES);
       for (int i = 0; i < n_tiles; ++i)
-        tma_load_3d(sbase + OFF_Q + i * TILE_BYTES, &tmap_q, bar(BAR_Q), 0, q0 + i * BM, b * p.H + h);
+        tma_load_3d(sbase + OFF_Q + i * Q_BYTES, &tmap_q, bar(BAR_Q), 0, q0 + i * BM, b * p.H + h);
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % STAGES;
@@ -384,9 +393,9 @@ __global__ void __launch_bounds__(core::THREADS, 1)
                             0x100u | st);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * TILE_BYTES);
-        tma_load_3d(sbase + OFF_K + st * TILE_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, b * p.H + h);
-        tma_load_4d(sbase + OFF_V + st * TILE_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+        mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * KV_BYTES);
+        tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, b * p.H + h);
+        tma_load_4d(sbase + OFF_V + st * KV_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
         ++issued[st];
       }
       if (!ok) {
@@ -399,63 +408,57 @@ __global__ void __launch_bounds__(core::THREADS, 1)
     }
   } else if (warp == 1 || warp == 2) {
     // ------------------------------------------------------------ MMA issuers
-    // Warp 1 issues every MMA of Q tile 0, warp 2 those of Q tile 1: one
-    // thread can issue a tcgen05.mma only every ~45-50 cycles, so the two
-    // tiles' instruction streams go out in parallel.  Within a tile the order
-    // PV(j-1), S(j) is one thread's program order.
     const int i = warp - 1;
     if (lane == 0 && !skip && i < n_tiles) {
       // Descriptors differ only in their start-address field (address >> 4).
-      const uint64_t dq = smem_desc_sw128(sbase + OFF_Q + i * TILE_BYTES, 16, 1024);
+      const uint64_t dq = smem_desc_sw128(sbase + OFF_Q + i * Q_BYTES, 16, 1024);
       const uint64_t dk = smem_desc_sw128(sbase + OFF_K, 16, 1024);
-      const uint64_t dv = smem_desc_sw128(sbase + OFF_V, 16384, 1024);
-      const uint32_t t_tile = tmem + i * TILE_COLS;
-      auto issue_s = [&](int st) {
-        const uint64_t k = dk + st * (TILE_BYTES >> 4);
+      const uint32_t t_s = tmem + i * 2 * BN, t_o = tmem + COL_O + i * NV;
+      auto issue_s = [&](int jj) {    // S(jj) into buffer jj % 2 from key stage jj % STAGES
+        const uint64_t k = dk + (jj % STAGES) * (KV_BYTES >> 4);
+        const uint32_t d = t_s + (jj & 1) * BN;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_ss(t_tile, dq + 2 * kk, k + 2 * kk, IDESC_QK, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) mma_ss(d, dq + 2 * kk, k + 2 * kk, IDESC_QK, kk > 0);
       };
-      // Key half hh: P at columns 64 hh .. of the tile's S (32 columns for 64
-      // keys), V rows 64 hh .. of the stage, accumulator O_i,hh.
-      auto issue_pv = [&](int st, bool acc) {
-        const uint64_t v = dv + st * (TILE_BYTES >> 4);
+      auto issue_pv = [&](int jj) {   // O += P(jj) V(jj), P in buffer jj % 2 (64 keys = 32 columns)
+        // Second MN atom (columns 64-79) = the ones tile: LBO is its distance
+        // from this stage's V tile.
+        const uint32_t v_addr = sbase + OFF_V + (jj % STAGES) * KV_BYTES;
+        const uint64_t v = smem_desc_sw128(v_addr, sbase + OFF_ONES - v_addr, 1024);
+        const uint32_t a = t_s + (jj & 1) * BN;
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-#pragma unroll
-          for (int kk = 0; kk < HALF / 16; ++kk)
-            mma_ts(t_tile + COL_O + hh * D, t_tile + hh * HALF + kk * 8, v + (hh * (HALF / 16) + kk) * (2048 >> 4),
-                   IDESC_PV, (acc || kk > 0) ? 1u : 0u);
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(t_o, a + kk * 8, v + kk * (2048 >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bounded(bar(BAR_Q), 0, abort_flag, p.status, p.timeout_ns, 0x200u) &&
-                wait_bounded(bar(BAR_KV_FULL), 0, abort_flag, p.status, p.timeout_ns, 0x210u);
-      // Stagger the two tiles by about half a period: tile 1 starts once tile
-      // 0's first softmax is done, so the two softmax phases alternate.
+      bool ok = wait_bounded(bar(BAR_Q), 0, abort_flag, p.status, p.timeout_ns, 0x200u);
+      // Stagger the two tiles: tile 1 starts once tile 0's first softmax step
+      // is done, so the two softmax warpgroups run out of phase.
       if (ok && i == 1) ok = wait_bounded(bar(BAR_P_FULL + 0), 0, abort_flag, p.status, p.timeout_ns, 0x2F0u);
-      if (ok) {
-        tc_fence_after();
-        issue_s(0);
-        tc_commit(bar(BAR_S_FULL + i));
-      }
-      for (int j = 1; j < n_kv && ok; ++j) {
-        const int st = j % STAGES, stp = (j - 1) % STAGES;
-        ok = wait_bounded(bar(BAR_KV_FULL + st), (j / STAGES) & 1, abort_flag, p.status, p.timeout_ns,
-                          0x210u | st) &&
-             wait_bounded(bar(BAR_P_FULL + i), (j - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x220u | i);
+      for (int jj = 0; jj < 2 && jj < n_kv && ok; ++jj) {
+        ok = wait_bounded(bar(BAR_KV_FULL + jj), 0, abort_flag, p.status, p.timeout_ns, 0x210u | jj);
         if (!ok) break;
         tc_fence_after();
-        issue_pv(stp, j > 1);
-        issue_s(st);
-        tc_commit(bar(BAR_S_FULL + i));
-        tc_commit(bar(BAR_KV_EMPTY + stp));
+        issue_s(jj);
+        tc_commit(bar(BAR_S_FULL + i * 2 + jj));
       }
-      if (ok) {
-        const int jl = n_kv - 1, stl = jl % STAGES;
-        ok = wait_bounded(bar(BAR_P_FULL + i), jl & 1, abort_flag, p.status, p.timeout_ns, 0x230u | i);
-        if (ok) {
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int buf = j & 1;
+        ok = wait_bounded(bar(BAR_P_FULL + i * 2 + buf), (j >> 1) & 1, abort_flag, p.status, p.timeout_ns,
+                          0x220u | i);
+        if (!ok) break;
+        tc_fence_after();
+        issue_pv(j);
+        tc_commit(bar(BAR_PV_DONE + i));
+        if (j == n_kv - 1) tc_commit(bar(BAR_O_FINAL + i));
+        tc_commit(bar(BAR_KV_EMPTY + (j % STAGES)));
+        const int jn = j + 2;
+        if (jn < n_kv) {
+          ok = wait_bounded(bar(BAR_KV_FULL + (jn % STAGES)), (jn / STAGES) & 1, abort_flag, p.status,
+                            p.timeout_ns, 0x230u | i);
+          if (!ok) break;
           tc_fence_after();
-          issue_pv(stl, jl > 0);
-          tc_commit(bar(BAR_O_FINAL + i));
-          tc_commit(bar(BAR_KV_EMPTY + stl));
+          issue_s(jn);
+          tc_commit(bar(BAR_S_FULL + i * 2 + buf));
         }
       }
       if (!ok) {  // let every MMA already issued finish before TMEM is released
