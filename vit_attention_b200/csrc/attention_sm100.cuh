@@ -8,8 +8,7 @@
 // the three modes, only the workspace views and the output row map differ.)
 //
 // Keys are processed in steps of 64.  Every Q tile has two S buffers in
-// TMEM, so the tensor core computes S(j+2) while the softmax works on S(j)
-// and the softmax never waits for a QK^T product it could have had earlier.
+// TMEM, so the tensor core computes S(j+2) while the softmax works on S(j+1).
 //
 // Warp roles (384 threads, 12 warps):
 //   warp 0       TMA producer: both Q tiles once, then K/V tiles of 64 keys
@@ -20,35 +19,43 @@
 //                so the two tiles' streams go out from two threads.  Per step
 //                j a tile's stream is
 //                  O_i += P_i(j) [V_j | 1]  (M=128, N=80, K=16 x 4, P from TMEM)
-//                  S_i(j+2) = Q_i K_j+2^T   (M=128, N=64, K=16 x 4, into the S
-//                                            buffer P_i(j) came from)
+//                  S_i(j+2) = Q_i K_j+2^T   (M=128, N=64, K=16 x 4, Q from TMEM,
+//                                            into the S buffer P_i(j) came from)
+//                  commit -> S_FULL          (also covers PV(j))
 //                in program order, so S(j+2) overwrites P(j) only after PV(j).
+//                Q sits in TMEM so that a QK^T product reads only its 2 KB of
+//                K from shared memory: with Q read from shared memory too
+//                (6 KB per product) those products were bound by shared-memory
+//                bandwidth rather than by the tensor core.
 //                The B operand of PV is V_j followed by 16 columns of ones
 //                (a constant shared-memory tile), so columns 64-79 of O_i
 //                accumulate the row sums of P on the tensor core and the
 //                softmax threads never add their probabilities up.
 //   warp 3       idle.
 //   warps 4-11   softmax, one warpgroup per Q tile; thread r owns query row r
-//                (= TMEM lane r).  Per step it reads its 64 scores, keeps a
+//                (= TMEM lane r).  First it copies its row of Q from shared
+//                memory into TMEM.  Per step it reads its 64 scores, keeps a
 //                running reference max m in fp32, writes P = 2^(s - m) as
 //                bf16 over the first 32 columns of the S buffer, and rescales
 //                O (head dims and the sum column) in TMEM only when m grows by
 //                more than 8 (a factor of 256; below that the stale max is
 //                kept, which is exact because O and its sum column always
-//                share the same m).  A rescale first waits for the previous PV
-//                to complete.  A small share of the exponentials runs on the
-//                FMA pipe (a cubic for 2^f after an exponent split), the rest
-//                on the MUFU unit.
+//                share the same m).  A small share of the exponentials runs on
+//                the FMA pipe (a cubic for 2^f after an exponent split), the
+//                rest on the MUFU unit.  Seeing S(j) complete also tells the
+//                warpgroup that PV(j-2) is complete, so it releases K/V stage
+//                j-2 to the producer, and a rescale at step j waits for S(j+1)
+//                (issued after PV(j-1)) rather than for a barrier of its own.
 //                Epilogue: O[:, 0:64] / O[:, 64] -> bf16 -> out.
 //
 // The row sum is that of the bf16-rounded P that multiplies V, so numerator
 // and denominator see the same rounding.
 //
 // TMEM (512 columns allocated): S buffers of tile i at columns 128 i and
-// 128 i + 64, O_i at 256 + 80 i (80 columns).  Every mbarrier wait is bounded
-// (wait_bounded); on expiry the CTA records VGGT_ATTN_ERR_TIMEOUT in the
-// workspace status word, drains what it has in flight and exits without
-// writing its output tiles.
+// 128 i + 64, O_i at 256 + 80 i (80 columns), Q_i at 416 + 32 i.  Every
+// mbarrier wait is bounded (wait_bounded); on expiry the CTA records
+// VGGT_ATTN_ERR_TIMEOUT in the workspace status word, drains what it has in
+// flight and exits without writing its output tiles.
 #pragma once
 
 #include <cstdint>
@@ -85,7 +92,8 @@ enum {
   BAR_P_FULL = BAR_S_FULL + NQ * 2,     // [tile][buffer]
   BAR_PV_DONE = BAR_P_FULL + NQ * 2,    // [tile]
   BAR_O_FINAL = BAR_PV_DONE + NQ,       // [tile]
-  BAR_DRAIN = BAR_O_FINAL + NQ,         // [issuer]
+  BAR_Q_TMEM = BAR_O_FINAL + NQ,        // [tile]: Q copied into TMEM
+  BAR_DRAIN = BAR_Q_TMEM + NQ,          // [issuer]
   N_BARS = BAR_DRAIN + NQ
 };
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
@@ -95,6 +103,7 @@ constexpr int THREADS = 384;
 constexpr bool PERSISTENT = false;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t COL_O = 256;                       // O_i (80 columns) at 256 + 80 i
+constexpr uint32_t COL_Q = 416;                       // Q_i (64 dims as bf16 pairs) at 416 + 32 i
 constexpr float RESCALE_THRESHOLD = 8.0f;              // log2 units
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
 // PV has N = 80: the 64 head dims of V, then 16 columns of ones whose
@@ -189,7 +198,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 }
 
 // Softmax warpgroup role: warps 4-7 own Q tile 0, warps 8-11 Q tile 1.
-__device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem, uint32_t bar0,
+__device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t* smem, uint32_t tmem, uint32_t bar0,
                                              volatile int* abort_flag, int h, int b, int q0, int n_kv, int warp,
                                              int lane) {
   using namespace core;
@@ -202,7 +211,29 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
   const uint32_t o_addr = tmem + lane_base + COL_O + tile * NV;
   const PolyConsts pc = poly_consts();
   float m_run = -INFINITY;
-  bool ok = true;
+  // Q tile -> TMEM (A operand of the QK^T products: row r in lane r, dims
+  // (2c, 2c+1) in column c), so that those products read only K from shared
+  // memory.  The tile sits in shared memory with the 128-byte swizzle: 16-byte
+  // chunk c of row r is stored at chunk c ^ (r % 8).
+  bool ok = wait_bounded(bar(BAR_Q), 0, abort_flag, p.status, p.timeout_ns, 0x330u | tile);
+  ok = __all_sync(0xffffffffu, ok);
+  if (!ok) return;
+  {
+    const uint4* qrow = reinterpret_cast<const uint4*>(smem + OFF_Q + tile * Q_BYTES + row * 128);
+    uint32_t qr[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = qrow[c ^ (row & 7)];
+      qr[4 * c] = v.x;
+      qr[4 * c + 1] = v.y;
+      qr[4 * c + 2] = v.z;
+      qr[4 * c + 3] = v.w;
+    }
+    tmem_st32(tmem + lane_base + COL_Q + tile * (D / 2), qr);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar(BAR_Q_TMEM + tile));
+  }
   for (int j = 0; j < n_kv; ++j) {
     const int buf = j & 1;
     const uint32_t s_addr = s_base + buf * BN;
@@ -210,6 +241,9 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
                       0x300u | tile);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) break;
+    // S(j) completing means PV(j-2) (issued before it by the same thread)
+    // has completed too: K/V stage j-2 is no longer read by this tile.
+    if (j >= 2 && (threadIdx.x & 127) == 0) mbar_arrive(bar(BAR_KV_EMPTY + (j - 2) % STAGES));
     tc_fence_after();
     uint32_t sr[2][32];
     tmem_ld32(s_addr, sr[0]);
@@ -263,7 +297,13 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, uint32_t tmem,
     // completed), so PV_DONE is at most one phase behind.  Warp-uniform:
     // tcgen05.ld/st are warp-collective.
     if (__any_sync(0xffffffffu, move && j > 0)) {
-      ok = wait_bounded(bar(BAR_PV_DONE + tile), (j - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x310u | tile);
+      // PV(j-1) must be complete: S(j+1) was issued after it, so its
+      // completion says so; past the last S, PV_DONE (committed only when no
+      // S follows a PV, first for PV(n_kv-2)) does.
+      ok = (j + 1 < n_kv)
+               ? wait_bounded(bar(BAR_S_FULL + tile * 2 + ((j + 1) & 1)), ((j + 1) >> 1) & 1, abort_flag, p.status,
+                              p.timeout_ns, 0x310u | tile)
+               : wait_bounded(bar(BAR_PV_DONE + tile), 0, abort_flag, p.status, p.timeout_ns, 0x318u | tile);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       tc_fence_after();
@@ -341,7 +381,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
     mbar_init(bar(BAR_Q), 1);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(BAR_KV_FULL + s), 1);
-      mbar_init(bar(BAR_KV_EMPTY + s), n_tiles);   // one commit per MMA issuer
+      mbar_init(bar(BAR_KV_EMPTY + s), n_tiles);   // one arrival per Q tile's softmax warpgroup
     }
     for (int i = 0; i < NQ; ++i) {
       for (int buf = 0; buf < 2; ++buf) {
@@ -350,6 +390,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
       }
       mbar_init(bar(BAR_PV_DONE + i), 1);
       mbar_init(bar(BAR_O_FINAL + i), 1);
+      mbar_init(bar(BAR_Q_TMEM + i), 128);
       mbar_init(bar(BAR_DRAIN + i), 1);
     }
     fence_mbar_init();
@@ -373,7 +414,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
 
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    if (!skip && ((warp >> 2) - 1) < n_tiles) softmax_role(p, tmem, bar0, abort_flag, h, b, q0, n_kv, warp, lane);
+    if (!skip && ((warp >> 2) - 1) < n_tiles) softmax_role(p, smem, tmem, bar0, abort_flag, h, b, q0, n_kv, warp, lane);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
   }
@@ -411,14 +452,14 @@ __global__ void __launch_bounds__(core::THREADS, 1)
     const int i = warp - 1;
     if (lane == 0 && !skip && i < n_tiles) {
       // Descriptors differ only in their start-address field (address >> 4).
-      const uint64_t dq = smem_desc_sw128(sbase + OFF_Q + i * Q_BYTES, 16, 1024);
       const uint64_t dk = smem_desc_sw128(sbase + OFF_K, 16, 1024);
       const uint32_t t_s = tmem + i * 2 * BN, t_o = tmem + COL_O + i * NV;
-      auto issue_s = [&](int jj) {    // S(jj) into buffer jj % 2 from key stage jj % STAGES
+      const uint32_t t_q = tmem + COL_Q + i * (D / 2);
+      auto issue_s = [&](int jj) {    // S(jj) into buffer jj % 2 from key stage jj % STAGES, Q from TMEM
         const uint64_t k = dk + (jj % STAGES) * (KV_BYTES >> 4);
         const uint32_t d = t_s + (jj & 1) * BN;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) mma_ss(d, dq + 2 * kk, k + 2 * kk, IDESC_QK, kk > 0);
+        for (int kk = 0; kk < D / 16; ++kk) mma_ts(d, t_q + kk * 8, k + 2 * kk, IDESC_QK, kk > 0);
       };
       auto issue_pv = [&](int jj) {   // O += P(jj) V(jj), P in buffer jj % 2 (64 keys = 32 columns)
         // Second MN atom (columns 64-79) = the ones tile: LBO is its distance
@@ -430,7 +471,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
         for (int kk = 0; kk < BN / 16; ++kk)
           mma_ts(t_o, a + kk * 8, v + kk * (2048 >> 4), IDESC_PV, (jj > 0 || kk > 0) ? 1u : 0u);
       };
-      bool ok = wait_bounded(bar(BAR_Q), 0, abort_flag, p.status, p.timeout_ns, 0x200u);
+      bool ok = wait_bounded(bar(BAR_Q_TMEM + i), 0, abort_flag, p.status, p.timeout_ns, 0x200u);
       // Stagger the two tiles: tile 1 starts once tile 0's first softmax step
       // is done, so the two softmax warpgroups run out of phase.
       if (ok && i == 1) ok = wait_bounded(bar(BAR_P_FULL + 0), 0, abort_flag, p.status, p.timeout_ns, 0x2F0u);
@@ -443,22 +484,25 @@ __global__ void __launch_bounds__(core::THREADS, 1)
       }
       for (int j = 0; j < n_kv && ok; ++j) {
         const int buf = j & 1;
+        const int jn = j + 2;
+        // K/V of step j+2 first (normally long resident), so that nothing
+        // but the MMAs sits between P(j) arriving and S(j+2) being issued.
+        if (jn < n_kv) {
+          ok = wait_bounded(bar(BAR_KV_FULL + (jn % STAGES)), (jn / STAGES) & 1, abort_flag, p.status,
+                            p.timeout_ns, 0x230u | i);
+          if (!ok) break;
+        }
         ok = wait_bounded(bar(BAR_P_FULL + i * 2 + buf), (j >> 1) & 1, abort_flag, p.status, p.timeout_ns,
                           0x220u | i);
         if (!ok) break;
         tc_fence_after();
         issue_pv(j);
-        tc_commit(bar(BAR_PV_DONE + i));
-        if (j == n_kv - 1) tc_commit(bar(BAR_O_FINAL + i));
-        tc_commit(bar(BAR_KV_EMPTY + (j % STAGES)));
-        const int jn = j + 2;
         if (jn < n_kv) {
-          ok = wait_bounded(bar(BAR_KV_FULL + (jn % STAGES)), (jn / STAGES) & 1, abort_flag, p.status,
-                            p.timeout_ns, 0x230u | i);
-          if (!ok) break;
-          tc_fence_after();
           issue_s(jn);
-          tc_commit(bar(BAR_S_FULL + i * 2 + buf));
+          tc_commit(bar(BAR_S_FULL + i * 2 + buf));   // also covers PV(j)
+        } else {
+          tc_commit(bar(BAR_PV_DONE + i));
+          if (j == n_kv - 1) tc_commit(bar(BAR_O_FINAL + i));
         }
       }
       if (!ok) {  // let every MMA already issued finish before TMEM is released
