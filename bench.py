@@ -342,7 +342,7 @@ def run_ours(args):
     traffic = recorded_traffic()
     roofline = {"bound": "tensor", "achieved": core_tflops, "peak": peak, "unit": "TFLOP/s",
                 "frac": core_tflops / peak, "traffic": traffic,
-                "kernel": "vggt::attn_core_kernel", "kernel_ms": core_ms,
+                "kernel": "vggt::attn_core_kernel<CoreCfg<2>>", "kernel_ms": core_ms,
                 "peak_source": f"{peak_src} bf16_tflops_sustained (back-to-back launches, seconds long)",
                 "frac_of_burst_peak": core_tflops / peaks.get("bf16_tflops", peak),
                 "prologue_ms": pro_ms,

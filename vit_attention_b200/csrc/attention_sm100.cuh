@@ -1,6 +1,8 @@
 // Exact softmax attention core for head_dim 64 on sm_100a (tcgen05 + TMEM + TMA).
 //
-// One CTA computes two 128-query tiles (256 queries) of one (problem, head):
+// One CTA computes NQ 128-query tiles of one (problem, head) (NQ = 2 in
+// global and register mode; NQ = 1 with two CTAs per SM in frame mode, see
+// CoreCfg; the text below describes NQ = 2):
 //   O = softmax(Q K^T) V   over the problem's L keys.  Q arrives scaled by
 //   softmax_scale*log2(e) from the prologue, so scores are in base 2.
 // (VGGT-Omega Aggregator explainer, section 3: the frame / global / register
@@ -10,7 +12,7 @@
 // Keys are processed in steps of 64.  Every Q tile has two S buffers in
 // TMEM, so the tensor core computes S(j+2) while the softmax works on S(j+1).
 //
-// Warp roles (384 threads, 12 warps):
+// Warp roles (384 threads, 12 warps; 256 threads for NQ = 1):
 //   warp 0       TMA producer: both Q tiles once, then K/V tiles of 64 keys
 //                through an 8-stage shared-memory ring (128-byte swizzle, no
 //                multicast).
@@ -51,8 +53,9 @@
 // The row sum is that of the bf16-rounded P that multiplies V, so numerator
 // and denominator see the same rounding.
 //
-// TMEM (512 columns allocated): S buffers of tile i at columns 128 i and
-// 128 i + 64, O_i at 256 + 80 i (80 columns), Q_i at 416 + 32 i.  Every
+// TMEM (512 columns allocated, 256 for NQ = 1): S buffers of tile i at
+// columns 128 i and 128 i + 64, O_i at 128 NQ + 80 i (80 columns), Q_i after
+// the O accumulators (32 columns each).  Every
 // mbarrier wait is bounded (wait_bounded); on expiry the CTA records
 // VGGT_ATTN_ERR_TIMEOUT in the workspace status word, drains what it has in
 // flight and exits without writing its output tiles.
@@ -76,34 +79,9 @@ struct CoreParams {
 };
 
 namespace core {
-constexpr int BM = 128, BN = 64, D = 64, STAGES = 8, NQ = 2;
+constexpr int BM = 128, BN = 64, D = 64;
 constexpr int Q_BYTES = BM * D * 2;                    // 16 KB query tile
 constexpr int KV_BYTES = BN * D * 2;                   // 8 KB key or value tile
-constexpr int OFF_Q = 0;                               // NQ tiles
-constexpr int OFF_K = OFF_Q + NQ * Q_BYTES;
-constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-constexpr int OFF_ONES = OFF_V + STAGES * KV_BYTES;    // 64 x 64 bf16 ones: the PV product's extra columns
-constexpr int OFF_BAR = OFF_ONES + KV_BYTES;
-enum {
-  BAR_Q = 0,
-  BAR_KV_FULL = 1,
-  BAR_KV_EMPTY = BAR_KV_FULL + STAGES,
-  BAR_S_FULL = BAR_KV_EMPTY + STAGES,   // [tile][buffer]
-  BAR_P_FULL = BAR_S_FULL + NQ * 2,     // [tile][buffer]
-  BAR_PV_DONE = BAR_P_FULL + NQ * 2,    // [tile]
-  BAR_O_FINAL = BAR_PV_DONE + NQ,       // [tile]
-  BAR_Q_TMEM = BAR_O_FINAL + NQ,        // [tile]: Q copied into TMEM
-  BAR_DRAIN = BAR_Q_TMEM + NQ,          // [issuer]
-  N_BARS = BAR_DRAIN + NQ
-};
-constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
-constexpr int SMEM_BYTES = OFF_MISC + 16;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;          // slack to align the base to 1024 B
-constexpr int THREADS = 384;
-constexpr bool PERSISTENT = false;
-constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_O = 256;                       // O_i (80 columns) at 256 + 80 i
-constexpr uint32_t COL_Q = 416;                       // Q_i (64 dims as bf16 pairs) at 416 + 32 i
 constexpr float RESCALE_THRESHOLD = 8.0f;              // log2 units
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
 // PV has N = 80: the 64 head dims of V, then 16 columns of ones whose
@@ -113,14 +91,70 @@ constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, NV, 0, 1);  // V is MN-major (h
 // Exponentials of score pair q (0..31 in a row of a step) run on the FMA pipe
 // when bit (q % 8) of this mask is set, on the MUFU unit otherwise.
 constexpr uint32_t POLY_PAIR_MASK = 0x80u;
-// Register split (setmaxnreg): warpgroup 0 gives registers back, the two
-// softmax warpgroups take them; the sum never exceeds the launch allocation
-// (launch_core checks the compiled register count before every launch).
-constexpr int REGS_AT_LAUNCH = 168;
-constexpr int REGS_PRODUCER = 56;
-constexpr int REGS_SOFTMAX = 224;
-static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 256 <= REGS_AT_LAUNCH * THREADS, "register split too large");
 }  // namespace core
+
+// Per-CTA shape of the kernel.  NQ = 2: two 128-query tiles share every K/V
+// tile (one CTA per SM; global and register mode, whose key loops are long).
+// NQ = 1: one tile per CTA and two CTAs per SM (frame mode: 17 key steps per
+// tile, so a CTA's start and end are a large share of its life, and the other
+// CTA on the SM keeps the tensor core and the MUFU unit busy meanwhile).
+template <int NQ_>
+struct CoreCfg {
+  static constexpr int NQ = NQ_;
+  static constexpr int CTAS_PER_SM = NQ_ == 2 ? 1 : 2;
+  static constexpr int STAGES = NQ_ == 2 ? 8 : 5;
+  static constexpr int OFF_Q = 0;                                  // NQ tiles
+  static constexpr int OFF_K = OFF_Q + NQ * core::Q_BYTES;
+  static constexpr int OFF_V = OFF_K + STAGES * core::KV_BYTES;
+  static constexpr int OFF_ONES = OFF_V + STAGES * core::KV_BYTES; // 64 x 64 bf16 ones: the PV product's extra columns
+  static constexpr int OFF_BAR = OFF_ONES + core::KV_BYTES;
+  enum {
+    BAR_Q = 0,
+    BAR_KV_FULL = 1,
+    BAR_KV_EMPTY = BAR_KV_FULL + STAGES,
+    BAR_S_FULL = BAR_KV_EMPTY + STAGES,   // [tile][buffer]
+    BAR_P_FULL = BAR_S_FULL + NQ * 2,     // [tile][buffer]
+    BAR_PV_DONE = BAR_P_FULL + NQ * 2,    // [tile]
+    BAR_O_FINAL = BAR_PV_DONE + NQ,       // [tile]
+    BAR_Q_TMEM = BAR_O_FINAL + NQ,        // [tile]: Q copied into TMEM
+    BAR_DRAIN = BAR_Q_TMEM + NQ,          // [issuer]
+    N_BARS = BAR_DRAIN + NQ
+  };
+  static constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;          // tmem slot, abort flag
+  static constexpr int SMEM_BYTES = OFF_MISC + 16;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;           // slack to align the base to 1024 B
+  static constexpr int THREADS = 128 * (1 + NQ);                 // producer/issuer warpgroup + one per tile
+  // TMEM per tile i: S buffers at 128 i and 128 i + 64, O (80 columns) at
+  // COL_O + 80 i, Q (64 dims as bf16 pairs) at COL_Q + 32 i.
+  static constexpr uint32_t TMEM_COLS = NQ == 2 ? 512 : 256;
+  static constexpr uint32_t COL_O = 128 * NQ;
+  static constexpr uint32_t COL_Q = COL_O + core::NV * NQ;
+  static_assert(COL_Q + 32 * NQ <= TMEM_COLS, "TMEM layout");
+  // Register split (setmaxnreg): warpgroup 0 gives registers back, the
+  // softmax warpgroups take them; the sum never exceeds the launch allocation
+  // (the host checks the compiled register count before every launch).
+  static constexpr int REGS_AT_LAUNCH = NQ == 2 ? 168 : 128;
+  static constexpr int REGS_PRODUCER = 56;
+  static constexpr int REGS_SOFTMAX = NQ == 2 ? 224 : 200;
+  static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 128 * NQ <= REGS_AT_LAUNCH * THREADS, "register split too large");
+  static_assert(REGS_AT_LAUNCH * THREADS * CTAS_PER_SM <= 65536, "registers per SM");
+};
+
+// Local names for a configuration's constants inside the templated roles.
+#define VGGT_CORE_CFG_NAMES(C)                                                                          \
+  constexpr int NQ = C::NQ, STAGES = C::STAGES;                                                        \
+  constexpr int OFF_Q = C::OFF_Q, OFF_K = C::OFF_K, OFF_V = C::OFF_V, OFF_ONES = C::OFF_ONES;          \
+  constexpr int OFF_BAR = C::OFF_BAR, OFF_MISC = C::OFF_MISC;                                          \
+  constexpr uint32_t TMEM_COLS = C::TMEM_COLS, COL_O = C::COL_O, COL_Q = C::COL_Q;                      \
+  constexpr int REGS_SOFTMAX = C::REGS_SOFTMAX, REGS_PRODUCER = C::REGS_PRODUCER;                      \
+  constexpr int BAR_Q = C::BAR_Q, BAR_KV_FULL = C::BAR_KV_FULL, BAR_KV_EMPTY = C::BAR_KV_EMPTY;        \
+  constexpr int BAR_S_FULL = C::BAR_S_FULL, BAR_P_FULL = C::BAR_P_FULL, BAR_PV_DONE = C::BAR_PV_DONE;  \
+  constexpr int BAR_O_FINAL = C::BAR_O_FINAL, BAR_Q_TMEM = C::BAR_Q_TMEM, BAR_DRAIN = C::BAR_DRAIN;    \
+  (void)NQ; (void)STAGES; (void)OFF_Q; (void)OFF_K; (void)OFF_V; (void)OFF_ONES; (void)OFF_BAR;         \
+  (void)OFF_MISC; (void)TMEM_COLS; (void)COL_O; (void)COL_Q; (void)REGS_SOFTMAX; (void)REGS_PRODUCER;   \
+  (void)BAR_Q; (void)BAR_KV_FULL; (void)BAR_KV_EMPTY; (void)BAR_S_FULL; (void)BAR_P_FULL;               \
+  (void)BAR_PV_DONE; (void)BAR_O_FINAL; (void)BAR_Q_TMEM; (void)BAR_DRAIN
+
 
 struct PolyConsts {
   uint64_t shift2, c3, c2, c1, c0;   // each: the same fp32 constant in both halves
@@ -198,10 +232,12 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
 }
 
 // Softmax warpgroup role: warps 4-7 own Q tile 0, warps 8-11 Q tile 1.
+template <class C>
 __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t* smem, uint32_t tmem, uint32_t bar0,
                                              volatile int* abort_flag, int h, int b, int q0, int n_kv, int warp,
                                              int lane) {
   using namespace core;
+  VGGT_CORE_CFG_NAMES(C);
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int tile = (warp >> 2) - 1;
   const int quarter = warp & 3;              // TMEM lane quarter this warp may access
@@ -359,10 +395,12 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
   }
 }
 
-__global__ void __launch_bounds__(core::THREADS, 1)
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
     attn_core_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, const CoreParams p) {
   using namespace core;
+  VGGT_CORE_CFG_NAMES(C);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -374,7 +412,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.y, b = blockIdx.z;
   const int q0 = blockIdx.x * (NQ * BM);
-  const int n_tiles = (q0 + BM < p.L) ? 2 : 1;          // the second Q tile may lie past the end
+  const int n_tiles = (NQ > 1 && q0 + BM < p.L) ? 2 : 1;   // the second Q tile may lie past the end
   const int n_kv = (p.L + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
@@ -414,7 +452,7 @@ __global__ void __launch_bounds__(core::THREADS, 1)
 
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    if (!skip && ((warp >> 2) - 1) < n_tiles) softmax_role(p, smem, tmem, bar0, abort_flag, h, b, q0, n_kv, warp, lane);
+    if (!skip && ((warp >> 2) - 1) < n_tiles) softmax_role<C>(p, smem, tmem, bar0, abort_flag, h, b, q0, n_kv, warp, lane);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
   }

@@ -140,8 +140,7 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.ws_qk[1] = w.k;
   p.ws_v = w.v;
   p.status = w.status;
-  p.n_rows = g.n_tok * g.n_c * s->H;
-  p.S = s->S;
+  p.n_tok = static_cast<int>(g.n_tok);
   p.T = s->T;
   p.H = s->H;
   p.n_special = s->n_special;
@@ -150,24 +149,55 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.mode = mode;
   p.L = static_cast<int>(g.L);
   p.n_c = g.n_c;
+  p.div_nspec = vggt::make_fastdiv(static_cast<uint32_t>(s->n_special));
+  p.div_L = vggt::make_fastdiv(static_cast<uint32_t>(g.L));
+  p.div_T = vggt::make_fastdiv(static_cast<uint32_t>(s->T));
+  p.div_gw = vggt::make_fastdiv(static_cast<uint32_t>(s->grid_w > 0 ? s->grid_w : 1));
   p.eps = s->ln_eps;
   const double scale = s->softmax_scale > 0.f ? static_cast<double>(s->softmax_scale) : 1.0 / std::sqrt(64.0);
   p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
   p.rope_base = s->rope_base;
 
-  // One block per token (grid-stride over tokens, four at a time), at most
-  // 8 blocks per SM.
-  const int threads = 256;
-  long long blocks = g.n_tok;
-  const long long cap = 148LL * 8;
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
+  // One 8-lane group per head row of a token (a group loops over rows when a
+  // token has more than 48); as many blocks as fit on the device at once,
+  // each striding over the tokens four at a time.
+  const int ch = g.n_c * s->H;
+  const int threads = ch <= 48 ? 8 * ch : 384;
   const size_t smem = static_cast<size_t>(s->grid_h + s->grid_w) * 16 * sizeof(float2);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(vggt::qk_norm_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
+  int dev = 0, sms = 0, per_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, vggt::qk_norm_rope_kernel, threads, smem) !=
+          cudaSuccess || per_sm < 1)
+    return VGGT_ATTN_ERR_CUDA;
+  long long blocks = static_cast<long long>(sms) * per_sm;
+  if (blocks > g.n_tok) blocks = g.n_tok;
+  if (blocks < 1) blocks = 1;
   vggt::qk_norm_rope_kernel<<<static_cast<unsigned>(blocks), threads, smem, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+template <class C>
+int launch_core_cfg(const ModeGeometry& g, int H, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                    const vggt::CoreParams& p, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(vggt::attn_core_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC) !=
+      cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  // The kernel re-splits its registers between warpgroups (setmaxnreg); that
+  // split assumes the compiled per-thread count.  A build with fewer registers
+  // at launch would make the softmax warps wait forever for registers, so
+  // refuse to launch it.
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, vggt::attn_core_kernel<C>) != cudaSuccess || fa.numRegs < C::REGS_AT_LAUNCH)
+    return VGGT_ATTN_ERR_CUDA;
+  constexpr int rows_per_cta = vggt::core::BM * C::NQ;
+  const long long n_q = (g.L + rows_per_cta - 1) / rows_per_cta;
+  const dim3 grid(static_cast<unsigned>(n_q), static_cast<unsigned>(H), static_cast<unsigned>(g.B));
+  vggt::attn_core_kernel<C><<<grid, C::THREADS, C::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
@@ -208,32 +238,10 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   p.out = static_cast<uint16_t*>(out);
   p.status = w.status;
   p.timeout_ns = kDefaultTimeoutNs;
-  if (cudaFuncSetAttribute(vggt::attn_core_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           vggt::core::SMEM_ALLOC) != cudaSuccess)
-    return VGGT_ATTN_ERR_CUDA;
-  // The kernel re-splits its registers between warpgroups (setmaxnreg); that
-  // split assumes the compiled per-thread count.  A build with fewer registers
-  // at launch would make the softmax warps wait forever for registers, so
-  // refuse to launch it.
-  cudaFuncAttributes fa;
-  if (cudaFuncGetAttributes(&fa, vggt::attn_core_kernel) != cudaSuccess ||
-      fa.numRegs < vggt::core::REGS_AT_LAUNCH)
-    return VGGT_ATTN_ERR_CUDA;
-  constexpr int rows_per_unit = vggt::core::BM * vggt::core::NQ;
-  const long long n_qp = (g.L + rows_per_unit - 1) / rows_per_unit;
-  dim3 grid(static_cast<unsigned>(n_qp), static_cast<unsigned>(s->H), static_cast<unsigned>(g.B));
-  if (vggt::core::PERSISTENT) {
-    // One CTA per SM walks the work units (query pair x head x problem).
-    const long long n_units = n_qp * s->H * g.B;
-    int dev = 0, n_sm = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
-      return VGGT_ATTN_ERR_CUDA;
-    if (n_units > 0x7FFFFFFFLL) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
-    grid = dim3(static_cast<unsigned>(n_units < n_sm ? n_units : n_sm));
-  }
-  vggt::attn_core_kernel<<<grid, vggt::core::THREADS, vggt::core::SMEM_ALLOC, stream>>>(mq, mk, mv, p);
-  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+  // Frame mode: one query tile per CTA, two CTAs per SM; global and register
+  // mode: two query tiles per CTA sharing every K/V tile.
+  if (mode == VGGT_ATTN_FRAME) return launch_core_cfg<vggt::CoreCfg<1>>(g, s->H, mq, mk, mv, p, stream);
+  return launch_core_cfg<vggt::CoreCfg<2>>(g, s->H, mq, mk, mv, p, stream);
 }
 
 bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
