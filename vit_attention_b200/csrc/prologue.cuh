@@ -9,16 +9,18 @@
 //                           register: B = 1, L = S*n_special)
 //   v    : [L][H][64]      (register mode only: the gathered special tokens)
 //
-// HBM-bound: 8 threads own one 128-byte head row (16 bytes each).  A block
-// has one 8-lane group per head row of a token (n_c*H groups, n_c*H*128
-// contiguous bytes of qkv), so a group keeps the same (tensor, head) for all
-// the tokens it visits and holds that row's gamma/beta in registers; each
-// lane keeps four tokens' loads in flight.  The LayerNorm reductions are 3
-// shuffles inside the 8-lane group, and a RoPE pair (j, j+16) sits in lanes g
-// and g^2 of the group.  Token -> (problem, position, frame slot) divisions
-// use a multiply-high by a precomputed reciprocal with one correction step.
-// The cos/sin table of every (row|col position, frequency) is built once per
-// block in fp64 and kept in shared memory as fp32.
+// HBM-bound: 4 threads own one 128-byte head row.  Lane l of a row's group
+// holds dims {b, .., b+7} and {b+16, .., b+23} with b = 32 (l / 2) + 8 (l % 2),
+// so both members of every RoPE pair (j, j+16) of its half sit in the lane
+// and the rotation needs no shuffle; the LayerNorm reductions are 2 shuffles
+// inside the 4-lane group.  A block has one group per head row of a token
+// (n_c*H groups, n_c*H*128 contiguous bytes of qkv), so a group keeps the same
+// (tensor, head) for all the tokens it visits and holds that row's gamma/beta
+// in registers; each lane keeps four tokens' loads in flight.  Token ->
+// (problem, position, frame slot) divisions use a multiply-high by a
+// precomputed reciprocal with one correction step.  The cos/sin table of
+// every (row|col position, frequency) is built once per block in fp64 and
+// kept in shared memory as fp32.
 #pragma once
 
 #include <cstdint>
@@ -51,6 +53,8 @@ __device__ __forceinline__ uint32_t fast_divmod(uint32_t n, const FastDiv& f, ui
   r = static_cast<uint32_t>(rr);
   return q;
 }
+
+constexpr int PRO_MAX_THREADS = 256;   // 4 lanes per head row: 64 rows per block at most
 
 struct PrologueParams {
   const uint16_t* qkv;
@@ -100,7 +104,7 @@ __device__ __forceinline__ PrologueToken prologue_token(const PrologueParams& p,
   return w;
 }
 
-__global__ void __launch_bounds__(384) qk_norm_rope_kernel(const PrologueParams p) {
+__global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const PrologueParams p) {
   extern __shared__ float2 rope_tab[];  // [(grid_h + grid_w) * 16]: (cos, sin)
   const int n_pos = p.grid_h + p.grid_w;
   for (int e = threadIdx.x; e < n_pos * 16; e += blockDim.x) {
@@ -117,98 +121,116 @@ __global__ void __launch_bounds__(384) qk_norm_rope_kernel(const PrologueParams 
   }
   __syncthreads();
 
-  const int g = threadIdx.x & 7;                    // lane inside the 8-lane row group
-  // Shuffles involve only the 8 lanes of one row group: the groups of a warp
+  const int l = threadIdx.x & 3;                    // lane inside the 4-lane row group
+  // Shuffles involve only the 4 lanes of one row group: the groups of a warp
   // may take different paths (v rows, loop tail).
-  const unsigned gmask = 0xFFu << (threadIdx.x & 24);
+  const unsigned gmask = 0xFu << (threadIdx.x & 28);
+  const int half = l >> 1;                          // 0: dims 0-31 rotate by row, 1: dims 32-63 by column
+  const int base = 32 * half + 8 * (l & 1);         // first dim of the lane's first run of 8
+  const int j0 = 8 * (l & 1);                       // RoPE frequency of the lane's first pair
   constexpr int TOKENS = 4;
   const int ch = p.n_c * p.H;
-  const int groups = blockDim.x >> 3;
-  for (int idx = threadIdx.x >> 3; idx < ch; idx += groups) {   // uniform over the 8-lane group
+  const int groups = blockDim.x >> 2;
+  for (int idx = threadIdx.x >> 2; idx < ch; idx += groups) {   // uniform over the 4-lane group
     const int c = idx / p.H, h = idx - c * p.H;
-    float gg[8], bb[8];
+    float ga[8], gb[8], ba[8], bb[8];               // gamma/beta of the lane's two runs
     if (c < 2) {
-      const float4* gm = reinterpret_cast<const float4*>(p.gamma[c] + h * 64 + g * 8);
-      const float4* bt = reinterpret_cast<const float4*>(p.beta[c] + h * 64 + g * 8);
-      const float4 g0 = __ldg(gm), g1 = __ldg(gm + 1), b0 = __ldg(bt), b1 = __ldg(bt + 1);
-      gg[0] = g0.x; gg[1] = g0.y; gg[2] = g0.z; gg[3] = g0.w;
-      gg[4] = g1.x; gg[5] = g1.y; gg[6] = g1.z; gg[7] = g1.w;
-      bb[0] = b0.x; bb[1] = b0.y; bb[2] = b0.z; bb[3] = b0.w;
-      bb[4] = b1.x; bb[5] = b1.y; bb[6] = b1.z; bb[7] = b1.w;
+      const float4* gm = reinterpret_cast<const float4*>(p.gamma[c] + h * 64 + base);
+      const float4* bt = reinterpret_cast<const float4*>(p.beta[c] + h * 64 + base);
+      const float4 g0 = __ldg(gm), g1 = __ldg(gm + 1), g2 = __ldg(gm + 4), g3 = __ldg(gm + 5);
+      const float4 b0 = __ldg(bt), b1 = __ldg(bt + 1), b2 = __ldg(bt + 4), b3 = __ldg(bt + 5);
+      ga[0] = g0.x; ga[1] = g0.y; ga[2] = g0.z; ga[3] = g0.w; ga[4] = g1.x; ga[5] = g1.y; ga[6] = g1.z; ga[7] = g1.w;
+      gb[0] = g2.x; gb[1] = g2.y; gb[2] = g2.z; gb[3] = g2.w; gb[4] = g3.x; gb[5] = g3.y; gb[6] = g3.z; gb[7] = g3.w;
+      ba[0] = b0.x; ba[1] = b0.y; ba[2] = b0.z; ba[3] = b0.w; ba[4] = b1.x; ba[5] = b1.y; ba[6] = b1.z; ba[7] = b1.w;
+      bb[0] = b2.x; bb[1] = b2.y; bb[2] = b2.z; bb[3] = b2.w; bb[4] = b3.x; bb[5] = b3.y; bb[6] = b3.z; bb[7] = b3.w;
     }
     const float mult = (c == 0) ? p.q_mult : 1.0f;
-    const long long row_src = static_cast<long long>(idx) * 64 + g * 8;        // (c, h) inside the token block
-    const long long row_dst = static_cast<long long>(h) * p.L * 64 + g * 8;    // head h of q/k
-    const int j0 = 8 * (g & 1);
-    const bool second = (g & 2) != 0;
-    const int half = g < 4 ? 0 : 1;                 // 0: row rotation (dims 0-31), 1: column rotation
+    const long long row_src = static_cast<long long>(idx) * 64 + base;         // (c, h) inside the token block
+    const long long row_dst = static_cast<long long>(h) * p.L * 64 + base;     // head h of q/k
     for (int i0 = blockIdx.x; i0 < p.n_tok; i0 += TOKENS * gridDim.x) {
       PrologueToken w[TOKENS];
-      uint4 raw[TOKENS];
+      uint4 ra[TOKENS], rb[TOKENS];
 #pragma unroll
       for (int k = 0; k < TOKENS; ++k) {
         const int ik = i0 + k * gridDim.x;
         w[k] = prologue_token(p, static_cast<uint32_t>(ik < p.n_tok ? ik : i0));
       }
 #pragma unroll
-      for (int k = 0; k < TOKENS; ++k) raw[k] = *reinterpret_cast<const uint4*>(p.qkv + w[k].src + row_src);
+      for (int k = 0; k < TOKENS; ++k) {
+        const uint16_t* src = p.qkv + w[k].src + row_src;
+        ra[k] = *reinterpret_cast<const uint4*>(src);
+        rb[k] = *reinterpret_cast<const uint4*>(src + 16);
+      }
 #pragma unroll
       for (int k = 0; k < TOKENS; ++k) {
         if (i0 + k * static_cast<int>(gridDim.x) >= p.n_tok) continue;
         if (c == 2) {   // register-mode v gather: plain copy
-          *reinterpret_cast<uint4*>(p.ws_v + w[k].dst_v + h * 64 + g * 8) = raw[k];
+          uint16_t* dst = p.ws_v + w[k].dst_v + h * 64 + base;
+          *reinterpret_cast<uint4*>(dst) = ra[k];
+          *reinterpret_cast<uint4*>(dst + 16) = rb[k];
           continue;
         }
-        float x[8];
-        const uint32_t wd[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+        float xa[8], xb[8];
+        const uint32_t wa[4] = {ra[k].x, ra[k].y, ra[k].z, ra[k].w};
+        const uint32_t wb[4] = {rb[k].x, rb[k].y, rb[k].z, rb[k].w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          x[2 * e] = __uint_as_float(wd[e] << 16);
-          x[2 * e + 1] = __uint_as_float(wd[e] & 0xFFFF0000u);
+          xa[2 * e] = __uint_as_float(wa[e] << 16);
+          xa[2 * e + 1] = __uint_as_float(wa[e] & 0xFFFF0000u);
+          xb[2 * e] = __uint_as_float(wb[e] << 16);
+          xb[2 * e + 1] = __uint_as_float(wb[e] & 0xFFFF0000u);
         }
-        // LayerNorm over the 64 values held by the 8-lane group (two passes).
+        // LayerNorm over the 64 values held by the 4-lane group (two passes).
         float sum = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) sum += x[e];
+        for (int e = 0; e < 8; ++e) sum += xa[e] + xb[e];
         sum += __shfl_xor_sync(gmask, sum, 1);
         sum += __shfl_xor_sync(gmask, sum, 2);
-        sum += __shfl_xor_sync(gmask, sum, 4);
         const float mean = sum * (1.0f / 64.0f);
         float sq = 0.f;
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          x[e] -= mean;
-          sq += x[e] * x[e];
+          xa[e] -= mean;
+          xb[e] -= mean;
+          sq += xa[e] * xa[e] + xb[e] * xb[e];
         }
         sq += __shfl_xor_sync(gmask, sq, 1);
         sq += __shfl_xor_sync(gmask, sq, 2);
-        sq += __shfl_xor_sync(gmask, sq, 4);
         const float rstd = rsqrtf(sq * (1.0f / 64.0f) + p.eps);
 #pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = x[e] * rstd * gg[e] + bb[e];
-        // 2D RoPE on patch tokens.  Lanes 0-3 hold dims 0-31 (row), 4-7 dims
-        // 32-63 (col); lanes with bit 1 clear hold the first member j of a
-        // pair (j, j+16), their partner is lane g^2.  The branch is uniform
-        // over the 8-lane group, the shuffles run in every lane of the group.
-        float partner[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) partner[e] = __shfl_xor_sync(gmask, x[e], 2);
+        for (int e = 0; e < 8; ++e) {
+          xa[e] = xa[e] * rstd * ga[e] + ba[e];
+          xb[e] = xb[e] * rstd * gb[e] + bb[e];
+        }
+        // 2D RoPE on patch tokens: pair (j, j+16) of the lane's half is
+        // (xa[e], xb[e]) with j = j0 + e.
         if (w[k].t >= p.n_special) {
           uint32_t pcol;
           const uint32_t prow = fast_divmod(static_cast<uint32_t>(w[k].t - p.n_special), p.div_gw, pcol);
           const int pos_idx = half == 0 ? static_cast<int>(prow) : p.grid_h + static_cast<int>(pcol);
+          const float4* cs4 = reinterpret_cast<const float4*>(rope_tab + pos_idx * 16 + j0);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float2 cs = rope_tab[pos_idx * 16 + j0 + e];
-            x[e] = second ? (x[e] * cs.x + partner[e] * cs.y) : (x[e] * cs.x - partner[e] * cs.y);
+          for (int e2 = 0; e2 < 4; ++e2) {
+            const float4 cs = cs4[e2];   // (cos, sin) of frequencies j0 + 2 e2 and j0 + 2 e2 + 1
+            const float a0 = xa[2 * e2], b0 = xb[2 * e2], a1 = xa[2 * e2 + 1], b1 = xb[2 * e2 + 1];
+            xa[2 * e2] = a0 * cs.x - b0 * cs.y;
+            xb[2 * e2] = b0 * cs.x + a0 * cs.y;
+            xa[2 * e2 + 1] = a1 * cs.z - b1 * cs.w;
+            xb[2 * e2 + 1] = b1 * cs.z + a1 * cs.w;
           }
         }
-        uint4 o;
-        o.x = pack_bf16x2(x[0] * mult, x[1] * mult);
-        o.y = pack_bf16x2(x[2] * mult, x[3] * mult);
-        o.z = pack_bf16x2(x[4] * mult, x[5] * mult);
-        o.w = pack_bf16x2(x[6] * mult, x[7] * mult);
-        *reinterpret_cast<uint4*>(p.ws_qk[c] + w[k].dst_qk + row_dst) = o;
+        uint4 oa, ob;
+        oa.x = pack_bf16x2(xa[0] * mult, xa[1] * mult);
+        oa.y = pack_bf16x2(xa[2] * mult, xa[3] * mult);
+        oa.z = pack_bf16x2(xa[4] * mult, xa[5] * mult);
+        oa.w = pack_bf16x2(xa[6] * mult, xa[7] * mult);
+        ob.x = pack_bf16x2(xb[0] * mult, xb[1] * mult);
+        ob.y = pack_bf16x2(xb[2] * mult, xb[3] * mult);
+        ob.z = pack_bf16x2(xb[4] * mult, xb[5] * mult);
+        ob.w = pack_bf16x2(xb[6] * mult, xb[7] * mult);
+        uint16_t* dst = p.ws_qk[c] + w[k].dst_qk + row_dst;
+        *reinterpret_cast<uint4*>(dst) = oa;
+        *reinterpret_cast<uint4*>(dst + 16) = ob;
       }
     }
   }

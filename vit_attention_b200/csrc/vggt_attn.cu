@@ -158,11 +158,11 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
   p.rope_base = s->rope_base;
 
-  // One 8-lane group per head row of a token (a group loops over rows when a
-  // token has more than 48); as many blocks as fit on the device at once,
+  // One 4-lane group per head row of a token (a group loops over rows when a
+  // token has more than 64); as many blocks as fit on the device at once,
   // each striding over the tokens four at a time.
   const int ch = g.n_c * s->H;
-  const int threads = ch <= 48 ? 8 * ch : 384;
+  const int threads = ch <= 64 ? 4 * ch : 256;
   const size_t smem = static_cast<size_t>(s->grid_h + s->grid_w) * 16 * sizeof(float2);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(vggt::qk_norm_rope_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
