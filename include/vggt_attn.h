@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VGGT_ATTN_ABI_VERSION 1
+#define VGGT_ATTN_ABI_VERSION 2
 
 /* Return codes (0 = success). */
 enum {
@@ -182,6 +182,55 @@ int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const void* qkv,
                       const float* q_gamma, const float* q_beta,
                       const float* k_gamma, const float* k_beta, void* out,
                       void* cuda_stream);
+
+/* ------------------------------------------------------------------------
+ * Projections either side of the attention core (VGGT-Omega Aggregator
+ * explainer, section 3: every attention block of the alternating-attention
+ * layer projects its C = H*64 channels to q, k and v, and its attention output
+ * back to C channels).  bf16 operands, fp32 accumulation on the tensor cores,
+ * bf16 results rounded to nearest even.  Weights use the nn.Linear layout
+ * [out_features][in_features]; biases are fp32 and may be NULL.
+ *
+ * vggt_linear: y[M][N] = x[M][K] . w[N][K]^T + bias[N].
+ *   M >= 1, N a multiple of 256, K a multiple of 64 (K, N <= 65536).
+ *   x, w, y, bias: 16-byte aligned; y must not overlap x or w.
+ *   `workspace` (>= 256 bytes, 256-byte aligned) receives the status word of
+ *   a device-side timeout (read with vggt_attn_read_status); it is not
+ *   cleared by this call.
+ *
+ * vggt_attn_qkv_proj: the QKV projection of a frame- or global-mode block with
+ * the prologue fused into it.  x is bf16 [S*T][C] (token features), w_qkv bf16
+ * [3C][C], b_qkv fp32 [3C] or NULL.  The q and k columns of every head go
+ * through the QK-LayerNorm, RoPE and softmax-scale step of vggt_attn_prologue
+ * in fp32 straight from the accumulator (no bf16 rounding of the projection
+ * before the LayerNorm) and land in `workspace`; the v columns are written to
+ * the v slot of qkv [S][T][3][H][64] (its q and k slots are not written).
+ * Afterwards vggt_attn_core(mode, shape, qkv, out, workspace, ...) computes
+ * the attention exactly as after vggt_attn_prologue.  Requires H a multiple
+ * of 4 (3C a multiple of 256); register mode is not supported
+ * (VGGT_ATTN_ERR_INVALID_ARG).  Clears the workspace status word.
+ *
+ * vggt_attn_block: one attention block, y = (attention(x W_qkv^T + b_qkv))
+ * W_out^T + b_out: vggt_attn_qkv_proj, vggt_attn_core into `attn` (bf16
+ * [S*T][C]), then vggt_linear with w_out [C][C], b_out [C] into y [S*T][C].
+ * `qkv` and `attn` are caller-provided scratch; y must not overlap x, qkv,
+ * attn or the workspace.  Modes and requirements as vggt_attn_qkv_proj.
+ *
+ * All three are asynchronous on `cuda_stream`, validate every argument before
+ * enqueueing anything and allocate nothing. */
+int vggt_linear(int M, int N, int K, const void* x, const void* w, const float* bias, void* y,
+                void* workspace, size_t workspace_bytes, void* cuda_stream);
+int vggt_attn_qkv_proj(int mode, const vggt_attn_shape* shape, const void* x,
+                       const void* w_qkv, const float* b_qkv,
+                       const float* q_gamma, const float* q_beta,
+                       const float* k_gamma, const float* k_beta, void* qkv,
+                       void* workspace, size_t workspace_bytes, void* cuda_stream);
+int vggt_attn_block(int mode, const vggt_attn_shape* shape, const void* x,
+                    const void* w_qkv, const float* b_qkv,
+                    const float* q_gamma, const float* q_beta,
+                    const float* k_gamma, const float* k_beta,
+                    const void* w_out, const float* b_out, void* qkv, void* attn, void* y,
+                    void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -49,3 +49,4 @@ from .attention import (  # noqa: F401
     register_tokens,
     resolved_scale,
 )
+from .projection import attention_block, linear, projected_qkv  # noqa: F401

@@ -87,18 +87,22 @@ def rope_2d(x: np.ndarray, row: np.ndarray, col: np.ndarray, base: float) -> np.
 def normalized_tokens(shape, inputs, flat_tokens: np.ndarray, which: Sequence[str] = ("q", "k", "v")):
     """QK-LayerNorm + RoPE'd q, k and raw v of the listed tokens.
 
-    ``flat_tokens`` are indices into the S*T token sequence (s*T + t).
+    ``flat_tokens`` are indices into the S*T token sequence (s*T + t).  q, k
+    and v come from ``inputs["qkv"]`` (bf16 bits ``[S, T, 3, H, 64]``), or from
+    ``inputs["qkv_f64"]`` (fp64, same shape) when the block's projection made them.
     Returns a dict of fp64 arrays ``[H, n, 64]`` for each name in ``which``.
     """
     flat_tokens = np.asarray(flat_tokens, dtype=np.int64)
     s, t = flat_tokens // shape.T, flat_tokens % shape.T
     is_patch, row, col = patch_row_col(t, shape.n_special, shape.grid_w)
-    qkv = inputs["qkv"]
     out = {}
     for c, name in enumerate(("q", "k", "v")):
         if name not in which:
             continue
-        x = bf16_to_f64(qkv[s, t, c])                        # [n, H, 64]
+        if "qkv_f64" in inputs:                              # projected in fp64 (attention block)
+            x = np.asarray(inputs["qkv_f64"][s, t, c], dtype=np.float64)
+        else:
+            x = bf16_to_f64(inputs["qkv"][s, t, c])          # [n, H, 64]
         if name != "v":
             x = layer_norm(x, inputs[f"{name}_gamma"][None], inputs[f"{name}_beta"][None], shape.ln_eps)
             rot = rope_2d(x, row[:, None], col[:, None], shape.rope_base)

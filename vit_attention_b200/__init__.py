@@ -63,6 +63,10 @@ _SIGNATURES = {
     "vggt_attn_error_string": (ctypes.c_char_p, [_int]),
     "vggt_attn_abi_version": (_int, []),
     "vggt_attn_noalloc": (_int, [_int, _shape_p, _vp, _fp, _fp, _fp, _fp, _vp, _vp]),
+    "vggt_linear": (_int, [_int, _int, _int, _vp, _vp, _fp, _vp, _vp, _sz, _vp]),
+    "vggt_attn_qkv_proj": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
+    "vggt_attn_block": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _fp, _vp, _vp, _vp, _vp, _sz,
+                               _vp]),
 }
 for _name, (_res, _args) in _SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -190,3 +194,31 @@ _ENTRY = {"frame": vggt_attn_frame, "global": vggt_attn_global, "register": vggt
 def attend(mode: str, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, stream=None):
     """Dispatch by mode name to vggt_attn_{frame,global,register}."""
     _ENTRY[mode](shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, None, stream)
+
+
+def vggt_linear(x, w, bias, y, workspace, workspace_bytes=None, stream=None):
+    """y[M][N] = x[M][K] . w[N][K]^T + bias[N] (bf16 tensors, fp32 bias or None)."""
+    M, K = x.shape[-2], x.shape[-1]
+    N = w.shape[0]
+    rc = _lib.vggt_linear(M, N, K, _ptr(x), _ptr(w), _ptr(bias), _ptr(y), _ptr(workspace),
+                          _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_linear")
+
+
+def vggt_attn_qkv_proj(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, workspace,
+                       workspace_bytes=None, stream=None):
+    mode = MODES.get(mode, mode)
+    rc = _lib.vggt_attn_qkv_proj(mode, ctypes.byref(make_shape(shape)), _ptr(x), _ptr(w_qkv), _ptr(b_qkv),
+                                 _ptr(q_gamma), _ptr(q_beta), _ptr(k_gamma), _ptr(k_beta), _ptr(qkv), _ptr(workspace),
+                                 _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_qkv_proj")
+
+
+def vggt_attn_block(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, w_out, b_out, qkv, attn, y,
+                    workspace, workspace_bytes=None, stream=None):
+    mode = MODES.get(mode, mode)
+    rc = _lib.vggt_attn_block(mode, ctypes.byref(make_shape(shape)), _ptr(x), _ptr(w_qkv), _ptr(b_qkv),
+                              _ptr(q_gamma), _ptr(q_beta), _ptr(k_gamma), _ptr(k_beta), _ptr(w_out), _ptr(b_out),
+                              _ptr(qkv), _ptr(attn), _ptr(y), _ptr(workspace), _nbytes(workspace, workspace_bytes),
+                              _stream(stream))
+    _check(rc, "vggt_attn_block")

@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "attention_sm100.cuh"
+#include "linear_sm100.cuh"
 #include "prologue.cuh"
 #include "vggt_attn.h"
 
@@ -433,3 +434,163 @@ extern "C" int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const v
                   cuda_stream);
 }
 
+
+// ---------------------------------------------------------------------------
+// Projections either side of the attention core: Y = X W^T + b, and the QKV
+// projection with the QK LayerNorm + RoPE in its epilogue.
+namespace {
+
+bool make_rows_map(CUtensorMap* map, const void* base, long long inner, long long rows, cuuint32_t box_rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(inner), static_cast<cuuint64_t>(rows), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(inner) * 2, static_cast<cuuint64_t>(inner) * 2 * rows};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(vggt::lin::BK), box_rows, 1};
+  return make_map(map, base, 3, dims, strides, box);
+}
+
+int check_linear_dims(long long M, long long N, long long K) {
+  if (M < 1 || N < vggt::lin::BN || K < vggt::lin::BK) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (N % vggt::lin::BN || K % vggt::lin::BK) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (M > (1LL << 30) || N > 65536 || K > 65536) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  return VGGT_ATTN_OK;
+}
+
+int launch_linear(vggt::LinearParams p, const void* x, const void* w, int grid_h, int grid_w, cudaStream_t stream) {
+  CUtensorMap mx, mw;
+  if (!make_rows_map(&mx, x, p.K, p.M, vggt::lin::BM) || !make_rows_map(&mw, w, p.K, p.N, vggt::lin::BN))
+    return VGGT_ATTN_ERR_CUDA;
+  const int smem = vggt::linear_smem_bytes(grid_h, grid_w);
+  if (cudaFuncSetAttribute(vggt::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return VGGT_ATTN_ERR_CUDA;
+  const long long tiles = ((p.M + vggt::lin::BM - 1) / vggt::lin::BM) * static_cast<long long>(p.N / vggt::lin::BN);
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);   // persistent: one CTA per SM
+  p.timeout_ns = kDefaultTimeoutNs;
+  vggt::linear_kernel<<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+int check_qkv_proj_args(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
+                        const float* gq, const float* bq, const float* gk, const float* bk, void* qkv, void* ws,
+                        size_t ws_bytes) {
+  if (mode != VGGT_ATTN_FRAME && mode != VGGT_ATTN_GLOBAL) return VGGT_ATTN_ERR_INVALID_ARG;
+  int rc = check_common(mode, s, qkv, ws, ws_bytes);
+  if (rc) return rc;
+  if (!x || !w || !gq || !bq || !gk || !bk) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w, 16) || (b && !aligned(b, 16)) || !aligned(gq, 16) || !aligned(bq, 16) ||
+      !aligned(gk, 16) || !aligned(bk, 16))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  const long long C = static_cast<long long>(s->H) * 64;
+  if ((rc = check_linear_dims(static_cast<long long>(s->S) * s->T, 3 * C, C))) return rc;
+  const size_t qkv_bytes = static_cast<size_t>(s->S) * s->T * 3 * C * 2;
+  const size_t x_bytes = static_cast<size_t>(s->S) * s->T * C * 2;
+  if (overlaps(qkv, qkv_bytes, x, x_bytes) || overlaps(ws, ws_bytes, x, x_bytes) ||
+      overlaps(qkv, qkv_bytes, w, static_cast<size_t>(3 * C * C * 2)))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
+                    const float* gq, const float* bq, const float* gk, const float* bk, void* qkv,
+                    const WorkspaceView& wv, cudaStream_t stream) {
+  const ModeGeometry g = geometry(s, mode);
+  vggt::LinearParams p{};
+  p.M = s->S * s->T;
+  p.N = 3 * s->H * 64;
+  p.K = s->H * 64;
+  p.bias = b;
+  p.status = wv.status;
+  p.zero_status = 1;
+  p.fused = 1;
+  p.ws_qk[0] = wv.q;
+  p.ws_qk[1] = wv.k;
+  p.qkv = static_cast<uint16_t*>(qkv);
+  p.gamma[0] = gq;
+  p.gamma[1] = gk;
+  p.beta[0] = bq;
+  p.beta[1] = bk;
+  p.H = s->H;
+  p.T = s->T;
+  p.L = static_cast<int>(g.L);
+  p.n_special = s->n_special;
+  p.grid_h = s->grid_h;
+  p.grid_w = s->grid_w > 0 ? s->grid_w : 1;
+  p.eps = s->ln_eps;
+  const double scale = s->softmax_scale > 0.f ? static_cast<double>(s->softmax_scale) : 1.0 / std::sqrt(64.0);
+  p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
+  p.rope_base = s->rope_base;
+  return launch_linear(p, x, w, s->grid_h, s->grid_w, stream);
+}
+
+}  // namespace
+
+extern "C" int vggt_linear(int M, int N, int K, const void* x, const void* w, const float* bias, void* y,
+                           void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_linear_dims(M, N, K);
+  if (rc) return rc;
+  if (!x || !w || !y || !workspace) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 16) || (bias && !aligned(bias, 16)) ||
+      !aligned(workspace, 256))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  if (workspace_bytes < vggt::kStatusBytes) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  const size_t y_bytes = static_cast<size_t>(M) * N * 2;
+  if (overlaps(y, y_bytes, x, static_cast<size_t>(M) * K * 2) || overlaps(y, y_bytes, w, static_cast<size_t>(N) * K * 2) ||
+      overlaps(y, y_bytes, workspace, vggt::kStatusBytes))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  vggt::LinearParams p{};
+  p.M = M;
+  p.N = N;
+  p.K = K;
+  p.bias = bias;
+  p.y = static_cast<uint16_t*>(y);
+  p.status = static_cast<int*>(workspace);
+  p.grid_h = 0;
+  p.grid_w = 1;
+  return launch_linear(p, x, w, 0, 0, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int vggt_attn_qkv_proj(int mode, const vggt_attn_shape* shape, const void* x, const void* w_qkv,
+                                  const float* b_qkv, const float* q_gamma, const float* q_beta, const float* k_gamma,
+                                  const float* k_beta, void* qkv, void* workspace, size_t workspace_bytes,
+                                  void* cuda_stream) {
+  int rc = check_qkv_proj_args(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, workspace,
+                               workspace_bytes);
+  if (rc) return rc;
+  if ((rc = check_device())) return rc;
+  return launch_qkv_proj(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv,
+                         workspace_view(shape, mode, workspace), static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const void* x, const void* w_qkv,
+                               const float* b_qkv, const float* q_gamma, const float* q_beta, const float* k_gamma,
+                               const float* k_beta, const void* w_out, const float* b_out, void* qkv, void* attn,
+                               void* y, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_qkv_proj_args(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, workspace,
+                               workspace_bytes);
+  if (rc) return rc;
+  if ((rc = check_core_args(mode, shape, qkv, attn, workspace, workspace_bytes))) return rc;
+  const long long M = static_cast<long long>(shape->S) * shape->T, C = static_cast<long long>(shape->H) * 64;
+  if (!w_out || !y) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(w_out, 16) || !aligned(y, 16) || (b_out && !aligned(b_out, 16))) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t y_bytes = static_cast<size_t>(M) * C * 2;
+  if (overlaps(y, y_bytes, attn, y_bytes) || overlaps(y, y_bytes, workspace, workspace_bytes) ||
+      overlaps(y, y_bytes, qkv, static_cast<size_t>(M) * 3 * C * 2) || overlaps(y, y_bytes, x, y_bytes))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const WorkspaceView wv = workspace_view(shape, mode, workspace);
+  if ((rc = launch_qkv_proj(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, wv, st))) return rc;
+  if ((rc = launch_core(mode, shape, qkv, attn, wv, st))) return rc;
+  vggt::LinearParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(C);
+  p.K = static_cast<int>(C);
+  p.bias = b_out;
+  p.y = static_cast<uint16_t*>(y);
+  p.status = wv.status;
+  p.grid_w = 1;
+  return launch_linear(p, attn, w_out, 0, 0, st);
+}

@@ -163,6 +163,29 @@ def make_random_inputs(shape: Shape, seed: int, lowrank: float = 0.0) -> Dict[st
     return inputs
 
 
+def make_block_inputs(shape: Shape, seed: int) -> Dict[str, np.ndarray]:
+    """Seeded inputs of one attention block on token features (projections included).
+
+    x: bf16 bits ``[S*T, C]`` ~ N(0, 1), C = H * head_dim (frame s from
+    ``default_rng([seed, 4, s])``); w_qkv ``[3C, C]`` and w_out ``[C, C]``: bf16
+    bits ~ N(0, 1/C), so projected values are ~ N(0, 1); b_qkv ``[3C]`` and b_out
+    ``[C]``: fp32 ~ 0.1 N(0, 1); q/k gamma/beta as for the attention core.
+    """
+    S, T, C = shape.S, shape.T, shape.H * shape.head_dim
+    out = make_norm_params(shape.H, seed, shape.head_dim)
+    x = np.empty((S * T, C), dtype=np.uint16)
+    for s in range(S):
+        x[s * T:(s + 1) * T] = f32_to_bf16_bits(
+            np.random.default_rng([seed, 4, s]).standard_normal((T, C), dtype=np.float32))
+    out["x"] = x
+    sd = np.float32(1.0 / np.sqrt(C))
+    out["w_qkv"] = f32_to_bf16_bits(np.random.default_rng([seed, 5]).standard_normal((3 * C, C), dtype=np.float32) * sd)
+    out["b_qkv"] = (0.1 * np.random.default_rng([seed, 6]).standard_normal(3 * C)).astype(np.float32)
+    out["w_out"] = f32_to_bf16_bits(np.random.default_rng([seed, 7]).standard_normal((C, C), dtype=np.float32) * sd)
+    out["b_out"] = (0.1 * np.random.default_rng([seed, 8]).standard_normal(C)).astype(np.float32)
+    return out
+
+
 def query_subset(n_queries: int, count: int, seed: int) -> np.ndarray:
     """Sorted seeded subset of query indices (all of them if count >= n)."""
     if count >= n_queries:
