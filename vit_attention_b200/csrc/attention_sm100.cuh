@@ -471,7 +471,7 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
       mbar_arrive_expect_tx(bar(BAR_Q), n_tiles * Q_BYTES);
       for (int i = 0; i < n_tiles; ++i)
-        tma_load_3d(sbase + OFF_Q + i * Q_BYTES, &tmap_q, bar(BAR_Q), 0, q0 + i * BM, b * p.H + h);
+        tma_load_3d(sbase + OFF_Q + i * Q_BYTES, &tmap_q, bar(BAR_Q), 0, q0 + i * BM, h * p.B + b);
       bool ok = true;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % STAGES;
@@ -481,7 +481,7 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * KV_BYTES);
-        tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, b * p.H + h);
+        tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
         tma_load_4d(sbase + OFF_V + st * KV_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
         ++issued[st];
       }

@@ -11,9 +11,11 @@
 //             columns of a 64-wide head slice of q or k go through the QK
 //             LayerNorm, the 2D RoPE and (q) the softmax scale in fp32 straight
 //             from the accumulator and land in the attention workspace in the
-//             core's layout [B][H][L][64]; v slices go to the v slot of
-//             qkv[S][T][3][H][64].  This replaces the separate prologue pass
-//             and its HBM round trip of q and k.
+//             core's layout (one [S*T][64] plane per head); v slices go to the
+//             v slot of qkv[S][T][3][H][64].  This replaces the separate
+//             prologue pass and its HBM round trip of q and k.
+// Every 64-column chunk of a tile is staged in shared memory (128-byte
+// swizzle) and written by one TMA store: whole lines, rows past M clipped.
 //
 // Persistent CTAs (one per SM) walk 128 x 256 output tiles (n fastest).  Warp
 // roles (256 threads):
@@ -23,8 +25,10 @@
 //                per k-step into one of two 256-column TMEM accumulators, so
 //                the epilogue of one tile overlaps the products of the next.
 //   warps 4-7    epilogue: thread r owns output row r of the tile (TMEM lane r);
-//                it reads 64 accumulator columns at a time, adds the bias and
-//                stores bf16 (or normalises/rotates, in the qkv epilogue).
+//                it reads 64 accumulator columns at a time, adds the bias,
+//                (qkv epilogue: normalises and rotates), and writes its 128-byte
+//                row of the chunk into the staging buffer; one thread stores
+//                the chunk with TMA.
 // Every mbarrier wait is bounded (wait_bounded); on expiry the CTA records
 // VGGT_ATTN_ERR_TIMEOUT in the status word and drains what it has in flight.
 #pragma once
@@ -41,13 +45,16 @@ constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_BAR = OFF_B + STAGES * B_BYTES;
+constexpr int OFF_STAGE = OFF_B + STAGES * B_BYTES;    // 128 x 64 bf16 output chunk (16 KB)
+constexpr int OFF_BAR = OFF_STAGE + BM * 128;
 enum {
   BAR_FULL = 0,
   BAR_EMPTY = BAR_FULL + STAGES,
   BAR_ACC_FULL = BAR_EMPTY + STAGES,   // [accumulator]
   BAR_ACC_EMPTY = BAR_ACC_FULL + 2,    // [accumulator]
-  BAR_DRAIN = BAR_ACC_EMPTY + 2,
+  BAR_STAGE_FULL = BAR_ACC_EMPTY + 2,  // every epilogue thread wrote its row of the chunk
+  BAR_STAGE_FREE = BAR_STAGE_FULL + 1, // the chunk's TMA store has read the buffer
+  BAR_DRAIN = BAR_STAGE_FREE + 1,
   N_BARS = BAR_DRAIN + 1
 };
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
@@ -61,19 +68,33 @@ constexpr int REGS_AT_LAUNCH = 168;
 struct LinearParams {
   int M, N, K;
   const float* bias;          // [N] or null
-  uint16_t* y;                // plain epilogue: [M][N]
   int* status;
   unsigned long long timeout_ns;
   int zero_status;            // clear the status word first (the first kernel of an attention block)
-  // qkv epilogue (fused == 1); N = 3 * H * 64, K = H * 64
+  // qkv epilogue (fused == 1); N = 3 * H * 64, K = H * 64; the destinations
+  // are the kernel's output tensor maps (v slot of qkv, q plane, k plane)
   int fused;
-  uint16_t* ws_qk[2];         // q, k destinations [B][H][L][64]
-  uint16_t* qkv;              // v destination: qkv[M][3][H][64]
   const float* gamma[2];
   const float* beta[2];
-  int H, T, L, n_special, grid_h, grid_w;
+  int H, T, n_special, grid_h, grid_w;
   float eps, q_mult, rope_base;
 };
+
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_4d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 __host__ __device__ inline int linear_smem_bytes(int grid_h, int grid_w) {
   return lin::OFF_ROPE + (grid_h + grid_w) * 16 * 8 + 1024;   // + slack to align the base to 1024 B
@@ -99,101 +120,152 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
       : "memory");
 }
 
-// Epilogue of one 128 x 256 tile: thread `row` owns output row m0 + row; acc
-// is its TMEM lane at the tile's accumulator.
-__device__ __forceinline__ void linear_epilogue(const LinearParams& p, uint32_t acc, int m0, int n0, int row,
-                                                const float2* rope_tab) {
-  const int m = m0 + row;
-  const bool valid = m < p.M;
+// Epilogue of one 128 x 256 tile: thread `row` owns output row m0 + row (its
+// TMEM lane at the tile's accumulator is `acc`).  Each 64-column chunk is
+// converted in registers, staged in shared memory and stored by the leader
+// thread with one TMA store; `chunk` counts the CTA's chunks (barrier phases).
+// Loads of bias, gamma and beta are issued a few at a time, so that the
+// chunk's 64 values are the only large live state.
+__device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t acc, int m0, int n0, int row,
+                                                bool leader, uint8_t* stage, uint32_t bar0, volatile int* abort_flag,
+                                                int& chunk, const CUtensorMap* to0, const CUtensorMap* to1,
+                                                const CUtensorMap* to2, const float2* rope_tab) {
+  using namespace lin;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  const int m = m0 + row;                 // rows past M compute garbage that TMA clips
 #pragma unroll 1
-  for (int ck = 0; ck < lin::BN / 64; ++ck) {
-    uint32_t r[64];
-    tmem_ld64(acc + ck * 64, r);
+  for (int ck = 0; ck < BN / 64; ++ck, ++chunk) {
+    uint32_t v[64];
+    tmem_ld64(acc + ck * 64, v);
     tmem_wait_ld();
     const int col0 = n0 + ck * 64;
-    float x[64];
+    if (p.bias) {
 #pragma unroll
-    for (int e = 0; e < 64; e += 4) {
-      const float4 bv = p.bias ? __ldg(reinterpret_cast<const float4*>(p.bias + col0 + e)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      x[e] = __uint_as_float(r[e]) + bv.x;
-      x[e + 1] = __uint_as_float(r[e + 1]) + bv.y;
-      x[e + 2] = __uint_as_float(r[e + 2]) + bv.z;
-      x[e + 3] = __uint_as_float(r[e + 3]) + bv.w;
+      for (int e = 0; e < 64; e += 4) {
+        const float4 bv = __ldg(reinterpret_cast<const float4*>(p.bias + col0 + e));
+        v[e] = __float_as_uint(__uint_as_float(v[e]) + bv.x);
+        v[e + 1] = __float_as_uint(__uint_as_float(v[e + 1]) + bv.y);
+        v[e + 2] = __float_as_uint(__uint_as_float(v[e + 2]) + bv.z);
+        v[e + 3] = __float_as_uint(__uint_as_float(v[e + 3]) + bv.w);
+      }
     }
     const int c = p.fused ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
-    if (!valid) continue;
-    if (c == 2) {
-      uint16_t* dst = (p.fused ? p.qkv : p.y) + static_cast<size_t>(m) * p.N + col0;
-#pragma unroll
-      for (int v = 0; v < 8; ++v) {
-        uint4 w;
-        w.x = pack_bf16x2(x[8 * v], x[8 * v + 1]);
-        w.y = pack_bf16x2(x[8 * v + 2], x[8 * v + 3]);
-        w.z = pack_bf16x2(x[8 * v + 4], x[8 * v + 5]);
-        w.w = pack_bf16x2(x[8 * v + 6], x[8 * v + 7]);
-        reinterpret_cast<uint4*>(dst)[v] = w;
-      }
-      continue;
-    }
-    // QK LayerNorm over the head's 64 values (biased variance, two passes).
     const int h = (col0 / 64) % p.H;
-    float sum = 0.f;
+    uint4 o[8];
+    if (c == 2) {
 #pragma unroll
-    for (int e = 0; e < 64; ++e) sum += x[e];
-    const float mean = sum * (1.0f / 64.0f);
-    float sq = 0.f;
+      for (int k = 0; k < 8; ++k) {
+        o[k].x = pack_bf16x2(__uint_as_float(v[8 * k]), __uint_as_float(v[8 * k + 1]));
+        o[k].y = pack_bf16x2(__uint_as_float(v[8 * k + 2]), __uint_as_float(v[8 * k + 3]));
+        o[k].z = pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]));
+        o[k].w = pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
+      }
+    } else {
+      // QK LayerNorm over the head's 64 values (biased variance, two passes;
+      // eight partial sums each, then a short tree).
+      float ps[8];
 #pragma unroll
-    for (int e = 0; e < 64; ++e) {
-      x[e] -= mean;
-      sq += x[e] * x[e];
-    }
-    const float rstd = rsqrtf(sq * (1.0f / 64.0f) + p.eps);
-    const float* gm = p.gamma[c] + h * 64;
-    const float* bt = p.beta[c] + h * 64;
+      for (int q = 0; q < 8; ++q) ps[q] = __uint_as_float(v[q]);
 #pragma unroll
-    for (int e = 0; e < 64; e += 4) {
-      const float4 g4 = __ldg(reinterpret_cast<const float4*>(gm + e));
-      const float4 b4 = __ldg(reinterpret_cast<const float4*>(bt + e));
-      x[e] = x[e] * rstd * g4.x + b4.x;
-      x[e + 1] = x[e + 1] * rstd * g4.y + b4.y;
-      x[e + 2] = x[e + 2] * rstd * g4.z + b4.z;
-      x[e + 3] = x[e + 3] * rstd * g4.w + b4.w;
-    }
-    // 2D RoPE on patch tokens: dims [0,32) by row, [32,64) by column, pairs (j, j+16).
-    const int t = m % p.T;
-    if (t >= p.n_special) {
-      const int pp = t - p.n_special;
-      const int prow = pp / p.grid_w, pcol = pp - prow * p.grid_w;
+      for (int e = 8; e < 64; ++e) ps[e & 7] += __uint_as_float(v[e]);
+      const float mean = (((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]))) * (1.0f / 64.0f);
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const float2* cs = rope_tab + (half == 0 ? prow : p.grid_h + pcol) * 16;
+      for (int q = 0; q < 8; ++q) ps[q] = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const float2 v = cs[j];
-          const float a = x[32 * half + j], b = x[32 * half + j + 16];
-          x[32 * half + j] = a * v.x - b * v.y;
-          x[32 * half + j + 16] = b * v.x + a * v.y;
+      for (int e = 0; e < 64; ++e) {
+        const float d = __uint_as_float(v[e]) - mean;
+        v[e] = __float_as_uint(d);
+        ps[e & 7] += d * d;
+      }
+      const float sq = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+      const float rstd = rsqrtf(sq * (1.0f / 64.0f) + p.eps);
+      const float mult = (c == 0) ? p.q_mult : 1.0f;
+      // Affine, then 2D RoPE on patch tokens (dims [0,32) by row, [32,64) by
+      // column, pairs (j, j+16)), then the q scale; one 32-dim half at a time.
+      const int t = m % p.T;
+      const bool patch = t >= p.n_special;
+      int prow = 0, pcol = 0;
+      if (patch) {
+        const int pp = t - p.n_special;
+        prow = pp / p.grid_w;
+        pcol = pp - prow * p.grid_w;
+      }
+      const float* gm = p.gamma[c] + h * 64;
+      const float* bt = p.beta[c] + h * 64;
+#pragma unroll
+      for (int hf = 0; hf < 2; ++hf) {
+        const float2* cs = rope_tab + (hf == 0 ? prow : p.grid_h + pcol) * 16;
+        float y[32];
+#pragma unroll
+        for (int j = 0; j < 16; j += 4) {
+          const int d0 = 32 * hf + j, d1 = d0 + 16;
+          const float4 g0 = __ldg(reinterpret_cast<const float4*>(gm + d0));
+          const float4 g1 = __ldg(reinterpret_cast<const float4*>(gm + d1));
+          const float4 b0 = __ldg(reinterpret_cast<const float4*>(bt + d0));
+          const float4 b1 = __ldg(reinterpret_cast<const float4*>(bt + d1));
+          const float ga[4] = {g0.x, g0.y, g0.z, g0.w}, gb[4] = {g1.x, g1.y, g1.z, g1.w};
+          const float ba[4] = {b0.x, b0.y, b0.z, b0.w}, bb[4] = {b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            float a = __uint_as_float(v[d0 + i]) * rstd * ga[i] + ba[i];
+            float bv = __uint_as_float(v[d1 + i]) * rstd * gb[i] + bb[i];
+            if (patch) {
+              const float2 w = cs[j + i];
+              const float a2 = a * w.x - bv * w.y;
+              bv = bv * w.x + a * w.y;
+              a = a2;
+            }
+            y[j + i] = a * mult;
+            y[j + i + 16] = bv * mult;
+          }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          o[4 * hf + k].x = pack_bf16x2(y[8 * k], y[8 * k + 1]);
+          o[4 * hf + k].y = pack_bf16x2(y[8 * k + 2], y[8 * k + 3]);
+          o[4 * hf + k].z = pack_bf16x2(y[8 * k + 4], y[8 * k + 5]);
+          o[4 * hf + k].w = pack_bf16x2(y[8 * k + 6], y[8 * k + 7]);
         }
       }
     }
-    const float mult = (c == 0) ? p.q_mult : 1.0f;
-    const int b = m / p.L, pos = m - b * p.L;
-    uint16_t* dst = p.ws_qk[c] + ((static_cast<size_t>(b) * p.H + h) * p.L + pos) * 64;
-#pragma unroll
-    for (int v = 0; v < 8; ++v) {
-      uint4 w;
-      w.x = pack_bf16x2(x[8 * v] * mult, x[8 * v + 1] * mult);
-      w.y = pack_bf16x2(x[8 * v + 2] * mult, x[8 * v + 3] * mult);
-      w.z = pack_bf16x2(x[8 * v + 4] * mult, x[8 * v + 5] * mult);
-      w.w = pack_bf16x2(x[8 * v + 6] * mult, x[8 * v + 7] * mult);
-      reinterpret_cast<uint4*>(dst)[v] = w;
+    // Stage the chunk: wait until the previous chunk's store has read the buffer.
+    if (chunk > 0) {
+      if (leader) {
+        bulk_wait_read_all();
+        mbar_arrive(bar(BAR_STAGE_FREE));
+      }
+      bool ok = wait_bounded(bar(BAR_STAGE_FREE), (chunk - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x540u);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) return false;
     }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(stage + row * 128 + ((k ^ (row & 7)) * 16)) = o[k];
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    mbar_arrive(bar(BAR_STAGE_FULL));
+    bool ok = true;
+    if (leader) {
+      ok = wait_bounded(bar(BAR_STAGE_FULL), chunk & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
+      if (ok) {
+        const uint32_t src = smem_addr(stage);
+        if (!p.fused)
+          tma_store_3d(to0, src, col0, m0, 0);          // y [M][N]
+        else if (c == 2)
+          tma_store_4d(to0, src, 0, h, 2, m0);          // v slot of qkv [M][3][H][64]
+        else
+          tma_store_3d(c == 0 ? to1 : to2, src, 0, m0, h);   // q or k plane of head h
+        bulk_commit();
+      }
+    }
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
   }
+  return true;
 }
 
 __global__ void __launch_bounds__(lin::THREADS, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
-                  const LinearParams p) {
+                  const __grid_constant__ CUtensorMap tmap_o0, const __grid_constant__ CUtensorMap tmap_o1,
+                  const __grid_constant__ CUtensorMap tmap_o2, const LinearParams p) {
   using namespace lin;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -217,6 +289,8 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
       mbar_init(bar(BAR_ACC_FULL + a), 1);
       mbar_init(bar(BAR_ACC_EMPTY + a), 128);
     }
+    mbar_init(bar(BAR_STAGE_FULL), 128);
+    mbar_init(bar(BAR_STAGE_FREE), 1);
     mbar_init(bar(BAR_DRAIN), 1);
     fence_mbar_init();
     *abort_flag = 0;
@@ -226,6 +300,11 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     }
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_w);
+    tma_prefetch_desc(&tmap_o0);
+    if (p.fused) {
+      tma_prefetch_desc(&tmap_o1);
+      tma_prefetch_desc(&tmap_o2);
+    }
   }
   if (p.fused) {
     const int n_pos = p.grid_h + p.grid_w;
@@ -314,8 +393,9 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     if (!skip) {
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
+      const bool leader = threadIdx.x == 128;
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
-      int lt = 0;
+      int lt = 0, chunk = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
         const int ab = lt & 1;
         bool ok = wait_bounded(bar(BAR_ACC_FULL + ab), (lt >> 1) & 1, abort_flag, p.status, p.timeout_ns,
@@ -324,10 +404,13 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-        linear_epilogue(p, tmem + lane_base + ab * BN, m0, n0, row, rope_tab);
+        ok = linear_epilogue(p, tmem + lane_base + ab * BN, m0, n0, row, leader, smem + OFF_STAGE, bar0, abort_flag,
+                             chunk, &tmap_o0, &tmap_o1, &tmap_o2, rope_tab);
         tc_fence_before();
         mbar_arrive(bar(BAR_ACC_EMPTY + ab));
+        if (!ok) break;
       }
+      if (leader) bulk_wait_all();   // the last stores have completed before the CTA exits
     }
   }
 

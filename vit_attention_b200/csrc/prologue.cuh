@@ -5,8 +5,9 @@
 // each 64-dim head vector (biased variance, per-head affine), rotates patch
 // tokens, multiplies q by softmax_scale*log2(e) (so the core works in base 2)
 // and writes bf16 into the workspace in the attention core's layout
-//   q, k : [B][H][L][64]   (frame: B = S, L = T; global: B = 1, L = S*T;
-//                           register: B = 1, L = S*n_special)
+//   q, k : [H][B][L][64]   (frame: B = S, L = T; global: B = 1, L = S*T;
+//                           register: B = 1, L = S*n_special), i.e. one
+//                           [B*L][64] plane per head in the mode's token order
 //   v    : [L][H][64]      (register mode only: the gathered special tokens)
 //
 // HBM-bound: 4 threads own one 128-byte head row.  Lane l of a row's group
@@ -99,7 +100,7 @@ __device__ __forceinline__ PrologueToken prologue_token(const PrologueParams& p,
   fast_divmod(flat, p.div_T, t);
   w.t = static_cast<int>(t);
   w.src = static_cast<long long>(flat) * 3 * p.H * 64;
-  w.dst_qk = (static_cast<long long>(b) * p.H * p.L + pos) * 64;
+  w.dst_qk = (static_cast<long long>(b) * p.L + pos) * 64;
   w.dst_v = static_cast<long long>(pos) * p.H * 64;
   return w;
 }
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
     }
     const float mult = (c == 0) ? p.q_mult : 1.0f;
     const long long row_src = static_cast<long long>(idx) * 64 + base;         // (c, h) inside the token block
-    const long long row_dst = static_cast<long long>(h) * p.L * 64 + base;     // head h of q/k
+    const long long row_dst = static_cast<long long>(h) * p.n_tok * 64 + base; // plane of head h
     for (int i0 = blockIdx.x; i0 < p.n_tok; i0 += TOKENS * gridDim.x) {
       PrologueToken w[TOKENS];
       uint4 ra[TOKENS], rb[TOKENS];

@@ -454,11 +454,15 @@ int check_linear_dims(long long M, long long N, long long K) {
   return VGGT_ATTN_OK;
 }
 
-int launch_linear(vggt::LinearParams p, const void* x, const void* w, int grid_h, int grid_w, cudaStream_t stream) {
+// Output maps: o0 = y [M][N] (plain) or the v slot of qkv [M][3][H][64]
+// (fused, as (64, H, 3, M)); o1, o2 = the q and k planes [H][M][64] (fused).
+int launch_linear(vggt::LinearParams p, const void* x, const void* w, const CUtensorMap& o0, const CUtensorMap& o1,
+                  const CUtensorMap& o2, int grid_h, int grid_w, cudaStream_t stream) {
   CUtensorMap mx, mw;
   if (!make_rows_map(&mx, x, p.K, p.M, vggt::lin::BM) || !make_rows_map(&mw, w, p.K, p.N, vggt::lin::BN))
     return VGGT_ATTN_ERR_CUDA;
   const int smem = vggt::linear_smem_bytes(grid_h, grid_w);
+  if (smem > 227 * 1024) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
   if (cudaFuncSetAttribute(vggt::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
   int dev = 0, sms = 0;
@@ -468,7 +472,7 @@ int launch_linear(vggt::LinearParams p, const void* x, const void* w, int grid_h
   const long long tiles = ((p.M + vggt::lin::BM - 1) / vggt::lin::BM) * static_cast<long long>(p.N / vggt::lin::BN);
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);   // persistent: one CTA per SM
   p.timeout_ns = kDefaultTimeoutNs;
-  vggt::linear_kernel<<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, p);
+  vggt::linear_kernel<<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, o0, o1, o2, p);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
@@ -504,16 +508,12 @@ int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const voi
   p.status = wv.status;
   p.zero_status = 1;
   p.fused = 1;
-  p.ws_qk[0] = wv.q;
-  p.ws_qk[1] = wv.k;
-  p.qkv = static_cast<uint16_t*>(qkv);
   p.gamma[0] = gq;
   p.gamma[1] = gk;
   p.beta[0] = bq;
   p.beta[1] = bk;
   p.H = s->H;
   p.T = s->T;
-  p.L = static_cast<int>(g.L);
   p.n_special = s->n_special;
   p.grid_h = s->grid_h;
   p.grid_w = s->grid_w > 0 ? s->grid_w : 1;
@@ -521,7 +521,23 @@ int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const voi
   const double scale = s->softmax_scale > 0.f ? static_cast<double>(s->softmax_scale) : 1.0 / std::sqrt(64.0);
   p.q_mult = static_cast<float>(scale * 1.4426950408889634);  // log2(e)
   p.rope_base = s->rope_base;
-  return launch_linear(p, x, w, s->grid_h, s->grid_w, stream);
+  CUtensorMap mv, mq, mk;
+  const long long M = p.M, H = s->H;
+  {
+    const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), 3, static_cast<cuuint64_t>(M)};
+    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(3 * H) * 128};
+    const cuuint32_t box[4] = {64, 1, 1, vggt::lin::BM};
+    if (!make_map(&mv, qkv, 4, dims, strides, box)) return VGGT_ATTN_ERR_CUDA;
+  }
+  {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(M), static_cast<cuuint64_t>(H)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(M) * 128};
+    const cuuint32_t box[3] = {64, vggt::lin::BM, 1};
+    if (!make_map(&mq, wv.q, 3, dims, strides, box) || !make_map(&mk, wv.k, 3, dims, strides, box))
+      return VGGT_ATTN_ERR_CUDA;
+  }
+  (void)g;
+  return launch_linear(p, x, w, mv, mq, mk, s->grid_h, s->grid_w, stream);
 }
 
 }  // namespace
@@ -545,11 +561,12 @@ extern "C" int vggt_linear(int M, int N, int K, const void* x, const void* w, co
   p.N = N;
   p.K = K;
   p.bias = bias;
-  p.y = static_cast<uint16_t*>(y);
   p.status = static_cast<int*>(workspace);
   p.grid_h = 0;
   p.grid_w = 1;
-  return launch_linear(p, x, w, 0, 0, static_cast<cudaStream_t>(cuda_stream));
+  CUtensorMap my;
+  if (!make_rows_map(&my, y, N, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
+  return launch_linear(p, x, w, my, my, my, 0, 0, static_cast<cudaStream_t>(cuda_stream));
 }
 
 extern "C" int vggt_attn_qkv_proj(int mode, const vggt_attn_shape* shape, const void* x, const void* w_qkv,
@@ -589,8 +606,9 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
   p.N = static_cast<int>(C);
   p.K = static_cast<int>(C);
   p.bias = b_out;
-  p.y = static_cast<uint16_t*>(y);
   p.status = wv.status;
   p.grid_w = 1;
-  return launch_linear(p, attn, w_out, 0, 0, st);
+  CUtensorMap my;
+  if (!make_rows_map(&my, y, C, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
+  return launch_linear(p, attn, w_out, my, my, my, 0, 0, st);
 }
