@@ -379,6 +379,9 @@ def run_ours(args):
     modes = {}
     if not args.no_modes:
         modes = mode_timings(V, device, stream)
+    blocks = {}
+    if not args.no_blocks:
+        blocks = block_timings(V, device, stream)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -398,9 +401,59 @@ def run_ours(args):
                 "parallelism": f"independent replicas x{world} (weak)"}),
             "pct_of_peak": 100.0 * value / world / peak,
             "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
-            "cpu_baseline": cpu}
+            "blocks": blocks, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def block_timings(V, device, stream):
+    """One attention block (QKV GEMM, QK-norm/RoPE prologue, attention core,
+    output projection; vggt_attn_block) on token features, for the S=100 global
+    and the S=500 frame workloads: ms per block and per stage, the GEMMs'
+    TFLOP/s, and the fused QKV projection (GEMM with the prologue in its
+    epilogue) for comparison (device-drawn inputs, random weights of the model's
+    shapes)."""
+    import torch
+    res = {}
+    g = torch.Generator(device=device)
+    g.manual_seed(4321)
+    for label, idx, mode in (("global_S100", 3, "global"), ("frame_S500", 4, "frame")):
+        shape = W.workload(idx).shape
+        M, C = shape.S * shape.T, shape.H * 64
+        x = torch.randn((M, C), generator=g, device=device).to(torch.bfloat16)
+        w_qkv = (torch.randn((3 * C, C), generator=g, device=device) / C ** 0.5).to(torch.bfloat16)
+        w_out = (torch.randn((C, C), generator=g, device=device) / C ** 0.5).to(torch.bfloat16)
+        b_qkv = 0.1 * torch.randn(3 * C, generator=g, device=device)
+        b_out = 0.1 * torch.randn(C, generator=g, device=device)
+        prm = {k: (1.0 if "gamma" in k else 0.0) + 0.1 * torch.randn((shape.H, 64), generator=g, device=device)
+               for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}
+        qkv = torch.empty((shape.S, shape.T, 3, shape.H, 64), dtype=torch.bfloat16, device=device)
+        attn = torch.empty((M, C), dtype=torch.bfloat16, device=device)
+        y = torch.empty((M, C), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(V.vggt_attn_workspace_size(shape, mode), dtype=torch.uint8, device=device)
+        gq, bq, gk, bk = prm["q_gamma"], prm["q_beta"], prm["k_gamma"], prm["k_beta"]
+        stages = {
+            "block": lambda: V.vggt_attn_block(mode, shape, x, w_qkv, b_qkv, gq, bq, gk, bk, w_out, b_out, qkv, attn,
+                                               y, ws, None, stream),
+            "qkv_gemm": lambda: V.vggt_linear(x, w_qkv, b_qkv, qkv.view(M, 3 * C), ws, None, stream),
+            "prologue": lambda: V.vggt_attn_prologue(mode, shape, qkv, gq, bq, gk, bk, ws, None, stream),
+            "core": lambda: V.vggt_attn_core(mode, shape, qkv, attn, ws, None, stream),
+            "out_proj": lambda: V.vggt_linear(attn, w_out, b_out, y, ws, None, stream),
+            "qkv_proj_fused": lambda: V.vggt_attn_qkv_proj(mode, shape, x, w_qkv, b_qkv, gq, bq, gk, bk, qkv, ws,
+                                                           None, stream),
+        }
+        entry = {}
+        for name, fn in stages.items():
+            for _ in range(2):
+                fn()
+            entry[name + "_ms"] = cuda_time_ms(fn, stream, 5 if mode == "global" else 10)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        entry["qkv_gemm_tflops"] = 2.0 * M * 3 * C * C / (entry["qkv_gemm_ms"] / 1000) / 1e12
+        entry["out_proj_tflops"] = 2.0 * M * C * C / (entry["out_proj_ms"] / 1000) / 1e12
+        entry["qkv_proj_fused_tflops"] = 2.0 * M * 3 * C * C / (entry["qkv_proj_fused_ms"] / 1000) / 1e12
+        res[label] = entry
+        del x, qkv, attn, y, ws
+    return res
 
 
 def mode_timings(V, device, stream):
@@ -446,6 +499,7 @@ def main():
     ap.add_argument("--workload", type=int, default=HEADLINE,
                     help="index of a global-mode workload (default: the S=100 headline; 2 = S=24 for profiling)")
     ap.add_argument("--no-modes", action="store_true")
+    ap.add_argument("--no-blocks", action="store_true", help="skip the attention-block (projections + core) timings")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -211,10 +211,13 @@ int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const void* qkv,
  * (VGGT_ATTN_ERR_INVALID_ARG).  Clears the workspace status word.
  *
  * vggt_attn_block: one attention block, y = (attention(x W_qkv^T + b_qkv))
- * W_out^T + b_out: vggt_attn_qkv_proj, vggt_attn_core into `attn` (bf16
- * [S*T][C]), then vggt_linear with w_out [C][C], b_out [C] into y [S*T][C].
- * `qkv` and `attn` are caller-provided scratch; y must not overlap x, qkv,
- * attn or the workspace.  Modes and requirements as vggt_attn_qkv_proj.
+ * W_out^T + b_out: vggt_linear of x into qkv (bf16 [S*T][3C]),
+ * vggt_attn_prologue, vggt_attn_core into `attn` (bf16 [S*T][C]), then
+ * vggt_linear with w_out [C][C], b_out [C] into y [S*T][C].  (The fused
+ * vggt_attn_qkv_proj does less memory traffic but its LayerNorm/RoPE epilogue
+ * sets its time; the unfused pair measured faster.)  `qkv` and `attn` are
+ * caller-provided scratch; y must not overlap x, qkv, attn or the workspace.
+ * Modes and requirements as vggt_attn_qkv_proj.
  *
  * All three are asynchronous on `cuda_stream`, validate every argument before
  * enqueueing anything and allocate nothing. */

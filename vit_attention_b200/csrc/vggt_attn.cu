@@ -599,7 +599,22 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
   if ((rc = check_device())) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
   const WorkspaceView wv = workspace_view(shape, mode, workspace);
-  if ((rc = launch_qkv_proj(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, wv, st))) return rc;
+  // QKV projection as a plain GEMM into qkv, then the prologue: measured
+  // faster than the fused projection (whose LayerNorm/RoPE epilogue, not its
+  // products, sets its time) on both the frame and the global workloads.
+  {
+    vggt::LinearParams pq{};
+    pq.M = static_cast<int>(M);
+    pq.N = static_cast<int>(3 * C);
+    pq.K = static_cast<int>(C);
+    pq.bias = b_qkv;
+    pq.status = wv.status;
+    pq.grid_w = 1;
+    CUtensorMap mqkv;
+    if (!make_rows_map(&mqkv, qkv, 3 * C, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
+    if ((rc = launch_linear(pq, x, w_qkv, mqkv, mqkv, mqkv, 0, 0, st))) return rc;
+  }
+  if ((rc = launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st))) return rc;
   if ((rc = launch_core(mode, shape, qkv, attn, wv, st))) return rc;
   vggt::LinearParams p{};
   p.M = static_cast<int>(M);
