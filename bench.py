@@ -406,6 +406,27 @@ def run_ours(args):
     return 0
 
 
+def linear_only(spec: str) -> int:
+    """vggt_linear on device-drawn bf16 operands, 3 warm-up + 3 calls, ms per call printed."""
+    import torch
+    import vit_attention_b200 as V
+    M, N, K = (int(v) for v in spec.split(","))
+    g = torch.Generator(device="cuda")
+    g.manual_seed(99)
+    x = torch.randn((M, K), generator=g, device="cuda").to(torch.bfloat16)
+    w = (torch.randn((N, K), generator=g, device="cuda") / K ** 0.5).to(torch.bfloat16)
+    b = 0.1 * torch.randn(N, generator=g, device="cuda")
+    y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    fn = lambda: V.vggt_linear(x, w, b, y, ws)
+    for _ in range(3):
+        fn()
+    ms = cuda_time_ms(fn, torch.cuda.current_stream(), 3)
+    assert V.vggt_attn_read_status(ws) == 0
+    print(json.dumps({"linear": [M, N, K], "ms": ms, "tflops": 2.0 * M * N * K / (ms / 1000) / 1e12}), flush=True)
+    return 0
+
+
 def block_timings(V, device, stream):
     """One attention block (QKV GEMM, QK-norm/RoPE prologue, attention core,
     output projection; vggt_attn_block) on token features, for the S=100 global
@@ -500,8 +521,12 @@ def main():
                     help="index of a global-mode workload (default: the S=100 headline; 2 = S=24 for profiling)")
     ap.add_argument("--no-modes", action="store_true")
     ap.add_argument("--no-blocks", action="store_true", help="skip the attention-block (projections + core) timings")
+    ap.add_argument("--linear-only", default=None, metavar="M,N,K",
+                    help="run vggt_linear on an M x N x K problem a few times and exit (a small case for ncu)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
+    if args.linear_only:
+        return linear_only(args.linear_only)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
