@@ -50,3 +50,4 @@ from .attention import (  # noqa: F401
     resolved_scale,
 )
 from .projection import attention_block, linear, projected_qkv  # noqa: F401
+from .sga import attn_global_sga, sga_kept_tokens  # noqa: F401
