@@ -235,6 +235,27 @@ int vggt_attn_block(int mode, const vggt_attn_shape* shape, const void* x,
                     const void* w_out, const float* b_out, void* qkv, void* attn, void* y,
                     void* workspace, size_t workspace_bytes, void* cuda_stream);
 
+/* ------------------------------------------------------------------------
+ * Subsampled global attention (AVGGT article, section B, point 2, "SGA"): an
+ * approximation of global mode that keeps every query but only a grid of
+ * keys.  Kept keys K: every camera/register token (t < n_special) of every
+ * frame and the patch tokens at (row, col) with row % s_h == 0 and
+ * col % s_w == 0 (one per s_h x s_w window).  Discarded set D: the other
+ * tokens.  Query i attends to K, to its own key when i is in D (the diagonal),
+ * and to the mean over D of the normalised, rotated keys and of the values,
+ * counted |D| - [i in D] times.  q/k normalisation, RoPE and the softmax scale
+ * are those of global mode; s_h = s_w = 1 gives global attention.
+ *
+ * vggt_attn_sga_workspace_size: bytes of workspace for (shape, s_h, s_w), or 0
+ * if invalid (s_h, s_w >= 1).
+ * vggt_attn_global_sga: arguments as vggt_attn_global plus s_h, s_w (1..1024);
+ * writes all of `out`; asynchronous, validates before enqueueing. */
+size_t vggt_attn_sga_workspace_size(const vggt_attn_shape* shape, int s_h, int s_w);
+int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s_w, const void* qkv,
+                         const float* q_gamma, const float* q_beta,
+                         const float* k_gamma, const float* k_beta, void* out,
+                         void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -67,6 +67,8 @@ _SIGNATURES = {
     "vggt_attn_qkv_proj": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
     "vggt_attn_block": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _fp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
+    "vggt_attn_sga_workspace_size": (_sz, [_shape_p, _int, _int]),
+    "vggt_attn_global_sga": (_int, [_shape_p, _int, _int, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -222,3 +224,16 @@ def vggt_attn_block(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_be
                               _ptr(qkv), _ptr(attn), _ptr(y), _ptr(workspace), _nbytes(workspace, workspace_bytes),
                               _stream(stream))
     _check(rc, "vggt_attn_block")
+
+
+def vggt_attn_sga_workspace_size(shape, s_h: int, s_w: int) -> int:
+    return _lib.vggt_attn_sga_workspace_size(ctypes.byref(make_shape(shape)), s_h, s_w)
+
+
+def vggt_attn_global_sga(shape, s_h, s_w, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, workspace_bytes=None,
+                         stream=None):
+    """Subsampled global attention: kept key grid s_h x s_w, diagonal, mean pair."""
+    rc = _lib.vggt_attn_global_sga(ctypes.byref(make_shape(shape)), s_h, s_w, _ptr(qkv), _ptr(q_gamma), _ptr(q_beta),
+                                   _ptr(k_gamma), _ptr(k_beta), _ptr(out), _ptr(workspace),
+                                   _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_global_sga")

@@ -67,8 +67,21 @@
 
 namespace vggt {
 
+// Extra inputs of subsampled global attention (SGA): the per-row diagonal
+// and mean-pair terms the epilogue adds to the attention over the kept keys.
+struct SgaParams {
+  const uint16_t* q_plane;   // normalised q of every token, [H][N][64] (as the core reads it)
+  const uint16_t* k_plane;   // normalised k of every token, [H][N][64]
+  const uint16_t* qkv;       // raw qkv [N][3][H][64] (v of the diagonal)
+  const float* sums;         // [2][H][64]: sums over the discarded tokens of k (0) and v (1)
+  int n_d;                   // number of discarded tokens |D|
+  float inv_nd;              // 1 / |D| (0 when D is empty)
+  int T, n_special, grid_w, s_h, s_w;
+};
+
 struct CoreParams {
-  int L;              // keys (and queries) per problem
+  int L;              // queries per problem (and keys, except in SGA)
+  int Lk;             // keys per problem
   int H;              // heads
   int B;              // problems
   int out_T;          // tokens per frame of `out`
@@ -76,6 +89,7 @@ struct CoreParams {
   uint16_t* out;      // bf16 [.][H][64]
   int* status;
   unsigned long long timeout_ns;
+  SgaParams sga;      // SGA configuration only
 };
 
 namespace core {
@@ -98,9 +112,10 @@ constexpr uint32_t POLY_PAIR_MASK = 0x80u;
 // NQ = 1: one tile per CTA and two CTAs per SM (frame mode: 17 key steps per
 // tile, so a CTA's start and end are a large share of its life, and the other
 // CTA on the SM keeps the tensor core and the MUFU unit busy meanwhile).
-template <int NQ_>
+template <int NQ_, bool SGA_ = false>
 struct CoreCfg {
   static constexpr int NQ = NQ_;
+  static constexpr bool SGA = SGA_;   // subsampled global attention epilogue
   static constexpr int CTAS_PER_SM = NQ_ == 2 ? 1 : 2;
   static constexpr int STAGES = NQ_ == 2 ? 8 : 5;
   static constexpr int OFF_Q = 0;                                  // NQ tiles
@@ -231,6 +246,81 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       : "memory");
 }
 
+// Subsampled global attention (AVGGT article, section B, point 2): query i
+// also sees its own key when that key was discarded (the diagonal) and the
+// mean of the discarded keys/values counted n_i = |D| - [i discarded] times.
+// Folds both into the row's accumulator `o` (64 head dims) and row sum `osum`,
+// which are relative to the reference max m (base-2 scores: q is pre-scaled).
+__device__ __forceinline__ float dot_bf16_row(const uint16_t* a, const float* b_f32, const uint16_t* b_bf16) {
+  const uint4* a4 = reinterpret_cast<const uint4*>(a);
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint4 w = a4[k];
+    const uint32_t wd[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float lo = __uint_as_float(wd[e] << 16), hi = __uint_as_float(wd[e] & 0xFFFF0000u);
+      const int d = 8 * k + 2 * e;
+      float blo, bhi;
+      if (b_f32) {
+        blo = b_f32[d];
+        bhi = b_f32[d + 1];
+      } else {
+        const uint32_t bw = reinterpret_cast<const uint32_t*>(b_bf16)[d >> 1];
+        blo = __uint_as_float(bw << 16);
+        bhi = __uint_as_float(bw & 0xFFFF0000u);
+      }
+      acc[e] += lo * blo + hi * bhi;
+    }
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+__device__ __forceinline__ void sga_extra_terms(const CoreParams& p, int h, int i, float m, uint32_t (&o)[2][32],
+                                                uint32_t& osum) {
+  const SgaParams& g = p.sga;
+  const int t = i % g.T;
+  bool kept = t < g.n_special;
+  if (!kept) {
+    const int pp = t - g.n_special;
+    const int prow = pp / g.grid_w, pcol = pp - prow * g.grid_w;
+    kept = (prow % g.s_h == 0) && (pcol % g.s_w == 0);
+  }
+  const bool diag = !kept;
+  const int n_mean = g.n_d - (diag ? 1 : 0);
+  if (!diag && n_mean <= 0) return;
+  const uint16_t* q = g.q_plane + (static_cast<size_t>(h) * p.L + i) * 64;
+  const float* ksum = g.sums + h * 64;
+  const float* vsum = g.sums + (p.H + h) * 64;
+  float m2 = m, s_d = 0.f, s_m = 0.f, lw = 0.f;
+  if (diag) {
+    s_d = dot_bf16_row(q, nullptr, g.k_plane + (static_cast<size_t>(h) * p.L + i) * 64);
+    m2 = fmaxf(m2, s_d);
+  }
+  if (n_mean > 0) {
+    s_m = dot_bf16_row(q, ksum, nullptr) * g.inv_nd;
+    lw = log2f(static_cast<float>(n_mean));
+    m2 = fmaxf(m2, s_m + lw);
+  }
+  const float a = exp2f(m - m2);
+  const float pd = diag ? exp2f(s_d - m2) : 0.f;
+  const float pm = n_mean > 0 ? exp2f(s_m + lw - m2) * g.inv_nd : 0.f;   // weight of the mean pair, per unit of vsum
+  const uint16_t* v = g.qkv + (static_cast<size_t>(i) * 3 + 2) * p.H * 64 + h * 64;
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+#pragma unroll
+    for (int e = 0; e < 32; e += 2) {
+      const int d = 32 * c + e;
+      const uint32_t vw = reinterpret_cast<const uint32_t*>(v)[d >> 1];
+      const float v0 = __uint_as_float(vw << 16), v1 = __uint_as_float(vw & 0xFFFF0000u);
+      o[c][e] = __float_as_uint(__uint_as_float(o[c][e]) * a + pd * v0 + pm * vsum[d]);
+      o[c][e + 1] = __float_as_uint(__uint_as_float(o[c][e + 1]) * a + pd * v1 + pm * vsum[d + 1]);
+    }
+  }
+  osum = __float_as_uint(__uint_as_float(osum) * a + pd + pm * static_cast<float>(g.n_d));
+}
+
 // Softmax warpgroup role: warps 4-7 own Q tile 0 (TILE = 0), warps 8-11 Q
 // tile 1 (TILE = 1).
 template <class C, int TILE>
@@ -286,7 +376,7 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     tmem_ld32(s_addr, sr[0]);
     tmem_ld32(s_addr + 32, sr[1]);
     tmem_wait_ld();
-    const int valid = p.L - j * BN;          // keys of this step that exist (>= BN except on the last)
+    const int valid = p.Lk - j * BN;         // keys of this step that exist (>= BN except on the last)
     if (valid < BN) {                        // last step only (uniform branch)
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -375,6 +465,7 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     tmem_wait_ld();
     const int i = q0 + tile * BM + row;
     if (i < p.L) {
+      if constexpr (C::SGA) sga_extra_terms(p, h, i, m_run, orr, osum);
       const float inv = 1.f / __uint_as_float(osum);
       const long long out_row = static_cast<long long>(b) * p.out_T +
                                 static_cast<long long>(i / p.out_group) * p.out_T + (i % p.out_group);
@@ -414,7 +505,7 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
   const int h = blockIdx.y, b = blockIdx.z;
   const int q0 = blockIdx.x * (NQ * BM);
   const int n_tiles = (NQ > 1 && q0 + BM < p.L) ? 2 : 1;   // the second Q tile may lie past the end
-  const int n_kv = (p.L + BN - 1) / BN;
+  const int n_kv = (p.Lk + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
     mbar_init(bar(BAR_Q), 1);

@@ -1,0 +1,77 @@
+// Subsampled global attention (AVGGT article, section B, point 2, "SGA"):
+// keys/values are subsampled on the patch grid (one token per s_h x s_w
+// window, every camera/register token kept), every query is kept, each token
+// keeps its diagonal, and one mean key/value pair stands in for the discarded
+// columns.  The QK-LayerNorm + RoPE prologue of global mode writes q and k of
+// every token; these two kernels then gather the kept keys/values into dense
+// arrays for the attention core and sum k and v over the discarded tokens
+// (the core's epilogue adds the diagonal and the mean pair per row).
+#pragma once
+
+#include <cstdint>
+
+#include "common.cuh"
+
+namespace vggt {
+
+struct SgaGeometry {
+  int N, Nk, H, T, n_special, grid_w, s_h, s_w, nw, kept_per_frame;
+};
+
+// Flat token index (s*T + t) of the r-th kept key: frame r / kept_per_frame;
+// inside it the n_special special tokens, then the kept patches row-major.
+__device__ __forceinline__ int sga_kept_token(const SgaGeometry& g, int r) {
+  const int s = r / g.kept_per_frame, u = r - s * g.kept_per_frame;
+  int t = u;
+  if (u >= g.n_special) {
+    const int k = u - g.n_special;
+    const int kr = k / g.nw, kc = k - kr * g.nw;
+    t = g.n_special + kr * g.s_h * g.grid_w + kc * g.s_w;
+  }
+  return s * g.T + t;
+}
+
+__device__ __forceinline__ bool sga_is_kept(const SgaGeometry& g, int flat) {
+  const int t = flat % g.T;
+  if (t < g.n_special) return true;
+  const int pp = t - g.n_special;
+  const int prow = pp / g.grid_w, pcol = pp - prow * g.grid_w;
+  return (prow % g.s_h == 0) && (pcol % g.s_w == 0);
+}
+
+// Kept keys (normalised k plane [H][N][64] -> [H][Nk][64]) and values
+// (qkv [N][3][H][64] -> [Nk][H][64]); one block per kept token, 16 bytes per thread.
+__global__ void __launch_bounds__(256) sga_gather_kernel(SgaGeometry g, const uint16_t* k_plane, const uint16_t* qkv,
+                                                         uint16_t* ks_plane, uint16_t* vs) {
+  for (int r = blockIdx.x; r < g.Nk; r += gridDim.x) {
+    const int flat = sga_kept_token(g, r);
+    for (int e = threadIdx.x; e < g.H * 8; e += blockDim.x) {
+      const int h = e >> 3, c = e & 7;
+      reinterpret_cast<uint4*>(ks_plane + (static_cast<size_t>(h) * g.Nk + r) * 64)[c] =
+          reinterpret_cast<const uint4*>(k_plane + (static_cast<size_t>(h) * g.N + flat) * 64)[c];
+      reinterpret_cast<uint4*>(vs + (static_cast<size_t>(r) * g.H + h) * 64)[c] =
+          reinterpret_cast<const uint4*>(qkv + ((static_cast<size_t>(flat) * 3 + 2) * g.H + h) * 64)[c];
+    }
+  }
+}
+
+// sums[0][h][d] += k over the discarded tokens, sums[1][h][d] += v; thread =
+// (h, d) = blockIdx.y * blockDim.x + threadIdx.x, blocks stride over tokens.
+__global__ void __launch_bounds__(256) sga_sum_kernel(SgaGeometry g, const uint16_t* k_plane, const uint16_t* qkv,
+                                                      float* sums) {
+  const int hd = blockIdx.y * blockDim.x + threadIdx.x;
+  if (hd >= g.H * 64) return;
+  const int h = hd >> 6, d = hd & 63;
+  float ak = 0.f, av = 0.f;
+  for (int tok = blockIdx.x; tok < g.N; tok += gridDim.x) {
+    if (sga_is_kept(g, tok)) continue;   // uniform over the block
+    const uint16_t kb = k_plane[(static_cast<size_t>(h) * g.N + tok) * 64 + d];
+    const uint16_t vb = qkv[((static_cast<size_t>(tok) * 3 + 2) * g.H + h) * 64 + d];
+    ak += __uint_as_float(static_cast<uint32_t>(kb) << 16);
+    av += __uint_as_float(static_cast<uint32_t>(vb) << 16);
+  }
+  atomicAdd(sums + hd, ak);
+  atomicAdd(sums + g.H * 64 + hd, av);
+}
+
+}  // namespace vggt

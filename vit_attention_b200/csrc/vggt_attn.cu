@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -12,6 +13,7 @@
 #include "attention_sm100.cuh"
 #include "linear_sm100.cuh"
 #include "prologue.cuh"
+#include "sga.cuh"
 #include "vggt_attn.h"
 
 namespace {
@@ -230,8 +232,9 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
       if (!make_map(&mv, vbase, 4, dims, strides, box)) return VGGT_ATTN_ERR_CUDA;
     }
   }
-  vggt::CoreParams p;
+  vggt::CoreParams p{};
   p.L = static_cast<int>(g.L);
+  p.Lk = static_cast<int>(g.L);
   p.H = s->H;
   p.B = static_cast<int>(g.B);
   p.out_T = s->T;
@@ -626,4 +629,129 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
   CUtensorMap my;
   if (!make_rows_map(&my, y, C, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
   return launch_linear(p, attn, w_out, my, my, my, 0, 0, st);
+}
+
+// ---------------------------------------------------------------------------
+// Subsampled global attention (AVGGT article, section B, point 2).
+namespace {
+
+struct SgaLayout {
+  vggt::SgaGeometry g;
+  WorkspaceView w;          // status, q plane, k plane (all tokens)
+  uint16_t* ks;             // kept keys [H][Nk][64]
+  uint16_t* vs;             // kept values [Nk][H][64]
+  float* sums;              // [2][H][64]
+  size_t bytes;
+};
+
+bool sga_layout(const vggt_attn_shape* s, int s_h, int s_w, void* ws, SgaLayout* out) {
+  if (s_h < 1 || s_w < 1) return false;
+  vggt::SgaGeometry g{};
+  g.N = s->S * s->T;
+  g.H = s->H;
+  g.T = s->T;
+  g.n_special = s->n_special;
+  g.grid_w = s->grid_w > 0 ? s->grid_w : 1;
+  g.s_h = s_h;
+  g.s_w = s_w;
+  const int nh = s->grid_h > 0 ? (s->grid_h + s_h - 1) / s_h : 0;
+  g.nw = s->grid_w > 0 ? (s->grid_w + s_w - 1) / s_w : 0;
+  g.kept_per_frame = s->n_special + nh * g.nw;
+  g.Nk = s->S * g.kept_per_frame;
+  if (g.Nk < 1) return false;
+  SgaLayout L{};
+  L.g = g;
+  L.w = workspace_view(s, VGGT_ATTN_GLOBAL, ws);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = L.w.bytes;
+  const size_t ks_bytes = align256(static_cast<size_t>(g.Nk) * g.H * 64 * 2);
+  L.ks = reinterpret_cast<uint16_t*>(base + off);
+  off += ks_bytes;
+  L.vs = reinterpret_cast<uint16_t*>(base + off);
+  off += ks_bytes;
+  L.sums = reinterpret_cast<float*>(base + off);
+  off += align256(static_cast<size_t>(2) * g.H * 64 * 4);
+  L.bytes = off;
+  *out = L;
+  return true;
+}
+
+}  // namespace
+
+extern "C" size_t vggt_attn_sga_workspace_size(const vggt_attn_shape* shape, int s_h, int s_w) {
+  if (check_shape(shape, VGGT_ATTN_GLOBAL) != VGGT_ATTN_OK) return 0;
+  SgaLayout L;
+  if (!sga_layout(shape, s_h, s_w, nullptr, &L)) return 0;
+  return L.bytes;
+}
+
+extern "C" int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s_w, const void* qkv,
+                                    const float* q_gamma, const float* q_beta, const float* k_gamma,
+                                    const float* k_beta, void* out, void* workspace, size_t workspace_bytes,
+                                    void* cuda_stream) {
+  int rc = check_shape(shape, VGGT_ATTN_GLOBAL);
+  if (rc) return rc;
+  if (s_h < 1 || s_w < 1 || s_h > 1024 || s_w > 1024) return VGGT_ATTN_ERR_INVALID_ARG;
+  const size_t need = vggt_attn_sga_workspace_size(shape, s_h, s_w);
+  if (need == 0) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  // The global-mode checks cover qkv, gamma/beta, out and their overlaps with
+  // the part of the workspace they see; the rest is checked here.
+  if ((rc = check_prologue_args(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace,
+                                workspace_bytes)))
+    return rc;
+  if ((rc = check_core_args(VGGT_ATTN_GLOBAL, shape, qkv, out, workspace, workspace_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  SgaLayout L;
+  sga_layout(shape, s_h, s_w, workspace, &L);
+  const vggt::SgaGeometry& g = L.g;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // 1. QK-LayerNorm + RoPE of every token (global mode: one [N][64] plane per head).
+  if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, L.w, st))) return rc;
+  // 2. Sums over the discarded tokens, and the kept keys/values gathered.
+  if (cudaMemsetAsync(L.sums, 0, static_cast<size_t>(2) * g.H * 64 * 4, st) != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+      return VGGT_ATTN_ERR_CUDA;
+    const unsigned ycount = static_cast<unsigned>((g.H * 64 + 255) / 256);
+    const unsigned xcount = static_cast<unsigned>(std::max(1, std::min(g.N, sms * 8 / static_cast<int>(ycount) + 1)));
+    vggt::sga_sum_kernel<<<dim3(xcount, ycount), 256, 0, st>>>(g, L.w.k, static_cast<const uint16_t*>(qkv), L.sums);
+    vggt::sga_gather_kernel<<<static_cast<unsigned>(std::min(g.Nk, sms * 16)), 256, 0, st>>>(
+        g, L.w.k, static_cast<const uint16_t*>(qkv), L.ks, L.vs);
+    if (cudaGetLastError() != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  }
+  // 3. Attention of every query over the kept keys, plus the per-row diagonal
+  //    and mean-pair terms in the epilogue.
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};
+    const cuuint32_t box_k[3] = {64, vggt::core::BN, 1};
+    const cuuint64_t dq[3] = {64, static_cast<cuuint64_t>(g.N), static_cast<cuuint64_t>(g.H)};
+    const cuuint64_t sq[2] = {128, static_cast<cuuint64_t>(g.N) * 128};
+    const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(g.Nk), static_cast<cuuint64_t>(g.H)};
+    const cuuint64_t sk[2] = {128, static_cast<cuuint64_t>(g.Nk) * 128};
+    if (!make_map(&mq, L.w.q, 3, dq, sq, box_q) || !make_map(&mk, L.ks, 3, dk, sk, box_k)) return VGGT_ATTN_ERR_CUDA;
+    const cuuint32_t box_v[4] = {64, 1, vggt::core::BN, 1};
+    const cuuint64_t dv[4] = {64, static_cast<cuuint64_t>(g.H), static_cast<cuuint64_t>(g.Nk), 1};
+    const cuuint64_t sv[3] = {128, static_cast<cuuint64_t>(g.H) * 128, static_cast<cuuint64_t>(g.Nk) * g.H * 128};
+    if (!make_map(&mv, L.vs, 4, dv, sv, box_v)) return VGGT_ATTN_ERR_CUDA;
+  }
+  vggt::CoreParams p{};
+  p.L = g.N;
+  p.Lk = g.Nk;
+  p.H = g.H;
+  p.B = 1;
+  p.out_T = shape->T;
+  p.out_group = g.N;
+  p.out = static_cast<uint16_t*>(out);
+  p.status = L.w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  const int n_d = g.N - g.Nk;
+  p.sga = {L.w.q, L.w.k, static_cast<const uint16_t*>(qkv), L.sums, n_d, n_d > 0 ? 1.0f / n_d : 0.0f,
+           g.T, g.n_special, g.grid_w, g.s_h, g.s_w};
+  ModeGeometry mg{1, g.N, g.N, 2};
+  return launch_core_cfg<vggt::CoreCfg<2, true>>(mg, g.H, mq, mk, mv, p, st);
 }
