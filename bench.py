@@ -382,6 +382,9 @@ def run_ours(args):
     blocks = {}
     if not args.no_blocks:
         blocks = block_timings(V, device, stream)
+    sga = {}
+    if not args.no_modes:
+        sga = sga_timings(V, device, stream, qkv, prm, out, ms / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -401,7 +404,7 @@ def run_ours(args):
                 "parallelism": f"independent replicas x{world} (weak)"}),
             "pct_of_peak": 100.0 * value / world / peak,
             "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
-            "blocks": blocks, "cpu_baseline": cpu}
+            "blocks": blocks, "sga": sga, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -425,6 +428,29 @@ def linear_only(spec: str) -> int:
     assert V.vggt_attn_read_status(ws) == 0
     print(json.dumps({"linear": [M, N, K], "ms": ms, "tflops": 2.0 * M * N * K / (ms / 1000) / 1e12}), flush=True)
     return 0
+
+
+def sga_timings(V, device, stream, qkv, prm, out, global_ms):
+    """Subsampled global attention on the headline workload (kept-key grid s x s):
+    ms per call, speedup over the exact global call, TFLOP/s over the kept keys."""
+    import torch
+    w = W.workload(HEADLINE)
+    shape = w.shape
+    res = {}
+    n = shape.S * shape.T
+    for s_ in (2, 3):
+        ws = torch.empty(V.vggt_attn_sga_workspace_size(shape, s_, s_), dtype=torch.uint8, device=device)
+        fn = lambda: V.vggt_attn_global_sga(shape, s_, s_, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"],
+                                            prm["k_beta"], out, ws, None, stream)
+        for _ in range(2):
+            fn()
+        t = cuda_time_ms(fn, stream, 5)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        nk = shape.S * (shape.n_special + ((shape.grid_h + s_ - 1) // s_) * ((shape.grid_w + s_ - 1) // s_))
+        res[f"grid_{s_}x{s_}"] = {"ms": t, "kept_keys": nk, "speedup_vs_global": global_ms / t,
+                                 "tflops_over_kept_keys": 4.0 * n * nk * 64 * shape.H / (t / 1000) / 1e12}
+        del ws
+    return res
 
 
 def block_timings(V, device, stream):
