@@ -464,7 +464,7 @@ def block_timings(V, device, stream):
     res = {}
     g = torch.Generator(device=device)
     g.manual_seed(4321)
-    for label, idx, mode in (("global_S100", 3, "global"), ("frame_S500", 4, "frame")):
+    for label, idx, mode in (("global_S100", 3, "global"), ("frame_S500", 4, "frame"), ("register_S500", 4, "register")):
         shape = W.workload(idx).shape
         M, C = shape.S * shape.T, shape.H * 64
         x = torch.randn((M, C), generator=g, device=device).to(torch.bfloat16)
@@ -489,17 +489,23 @@ def block_timings(V, device, stream):
             "qkv_proj_fused": lambda: V.vggt_attn_qkv_proj(mode, shape, x, w_qkv, b_qkv, gq, bq, gk, bk, qkv, ws,
                                                            None, stream),
         }
+        if mode == "register":   # the block runs on the gathered special tokens; time it whole
+            stages = {"block": stages["block"]}
         entry = {}
         for name, fn in stages.items():
             for _ in range(2):
                 fn()
             entry[name + "_ms"] = cuda_time_ms(fn, stream, 5 if mode == "global" else 10)
         assert V.vggt_attn_read_status(ws, stream) == 0
+        res[label] = entry
+        if mode == "register":
+            del x, qkv, attn, y, ws
+            continue
         entry["qkv_gemm_tflops"] = 2.0 * M * 3 * C * C / (entry["qkv_gemm_ms"] / 1000) / 1e12
         entry["out_proj_tflops"] = 2.0 * M * C * C / (entry["out_proj_ms"] / 1000) / 1e12
         entry["qkv_proj_fused_tflops"] = 2.0 * M * 3 * C * C / (entry["qkv_proj_fused_ms"] / 1000) / 1e12
-        res[label] = entry
         del x, qkv, attn, y, ws
+    res["layer_S500_register_plus_frame_block_ms"] = res["register_S500"]["block_ms"] + res["frame_S500"]["block_ms"]
     return res
 
 

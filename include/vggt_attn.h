@@ -217,7 +217,11 @@ int vggt_attn_noalloc(int mode, const vggt_attn_shape* shape, const void* qkv,
  * vggt_attn_qkv_proj does less memory traffic but its LayerNorm/RoPE epilogue
  * sets its time; the unfused pair measured faster.)  `qkv` and `attn` are
  * caller-provided scratch; y must not overlap x, qkv, attn or the workspace.
- * Modes and requirements as vggt_attn_qkv_proj.
+ * Requires H a multiple of 4.  Register mode (workspace sized for register
+ * mode; 3 n_special <= T): the block runs on the special tokens only -- their
+ * rows of x are gathered, projected, attend over each other (register
+ * attention), are projected back and scattered to their rows of y; patch
+ * rows of y are not written, and attn holds the compact intermediates.
  *
  * All three are asynchronous on `cuda_stream`, validate every argument before
  * enqueueing anything and allocate nothing. */

@@ -56,11 +56,21 @@ def _block_case(mode, shape, seed, count):
     qkv = torch.empty((shape.S, shape.T, 3, shape.H, 64), dtype=torch.bfloat16, device="cuda")
     attn = torch.empty((M, C), dtype=torch.bfloat16, device="cuda")
     y = torch.empty((M, C), dtype=torch.bfloat16, device="cuda")
+    sentinel = -7.0
+    y.fill_(sentinel)
     V.vggt_attn_block(mode, shape, dev["x"], dev["w_qkv"], dev["b_qkv"], dev["q_gamma"], dev["q_beta"],
                       dev["k_gamma"], dev["k_beta"], dev["w_out"], dev["b_out"], qkv, attn, y, ws)
     assert V.vggt_attn_read_status(ws) == 0
     q = query_sample(mode, shape, count, seed)
     idx = torch.as_tensor(q, device="cuda")
+    if mode == "register":
+        # patch rows untouched; special rows checked against the oracle block
+        patch = torch.ones(M, dtype=torch.bool, device="cuda")
+        patch[torch.as_tensor(O.register_tokens(shape), device="cuda")] = False
+        assert bool((y[patch] == sentinel).all())
+        want_y = O.attention_block(mode, shape, blk, q)
+        got_y = y.index_select(0, idx).float().cpu().numpy().astype(np.float64)
+        return assert_close(got_y, want_y, f"block output {mode} {shape}")
     # the attention output between the projections
     inputs = {"qkv_f64": O.projected_qkv(shape, blk)}
     inputs.update({k: blk[k] for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")})
@@ -72,12 +82,12 @@ def _block_case(mode, shape, seed, count):
     return assert_close(got_y, want_y, f"block output {mode} {shape}")
 
 
-@pytest.mark.parametrize("mode", ["frame", "global"])
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
 def test_block_small_matches_oracle(mode):
     _block_case(mode, W.workload(0).shape, 31, 1 << 62)
 
 
-@pytest.mark.parametrize("mode", ["frame", "global"])
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
 def test_block_ragged_matches_oracle(mode):
     # 3 frames of 1031 tokens: 128-row tiles straddle frame boundaries.
     _block_case(mode, W.Shape(S=3, T=1031, H=16, n_special=17, grid_h=26, grid_w=39), 32, 512)

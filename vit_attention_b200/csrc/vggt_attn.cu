@@ -584,51 +584,106 @@ extern "C" int vggt_attn_qkv_proj(int mode, const vggt_attn_shape* shape, const 
                          workspace_view(shape, mode, workspace), static_cast<cudaStream_t>(cuda_stream));
 }
 
+namespace {
+
+// Rows of the special tokens of every frame: compact row r <-> token row
+// (r / n_special) * T + r % n_special.  to_compact: token rows -> compact rows.
+__global__ void __launch_bounds__(128) special_rows_kernel(const uint4* src, uint4* dst, int n_rows, int row_vec,
+                                                           int n_special, int T, int to_compact) {
+  for (int r = blockIdx.x; r < n_rows; r += gridDim.x) {
+    const long long tok = static_cast<long long>(r / n_special) * T + r % n_special;
+    const long long from = to_compact ? tok : r, to = to_compact ? r : tok;
+    for (int e = threadIdx.x; e < row_vec; e += blockDim.x)
+      dst[to * row_vec + e] = src[from * row_vec + e];
+  }
+}
+
+int launch_special_rows(const void* src, void* dst, int n_rows, long long row_bytes, int n_special, int T,
+                        bool to_compact, cudaStream_t st) {
+  const int grid = n_rows < 4096 ? n_rows : 4096;
+  special_rows_kernel<<<grid, 128, 0, st>>>(static_cast<const uint4*>(src), static_cast<uint4*>(dst), n_rows,
+                                            static_cast<int>(row_bytes / 16), n_special, T, to_compact ? 1 : 0);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+int launch_linear_plain(const void* x, const void* w, const float* b, void* y, long long M, long long N, long long K,
+                        int* status, cudaStream_t st) {
+  vggt::LinearParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.bias = b;
+  p.status = status;
+  p.grid_w = 1;
+  CUtensorMap my;
+  if (!make_rows_map(&my, y, N, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
+  return launch_linear(p, x, w, my, my, my, 0, 0, st);
+}
+
+int check_block_args(int mode, const vggt_attn_shape* s, const void* x, const void* w_qkv, const float* b_qkv,
+                     const float* gq, const float* bq, const float* gk, const float* bk, const void* w_out,
+                     const float* b_out, void* qkv, void* attn, void* y, void* ws, size_t ws_bytes) {
+  int rc = check_prologue_args(mode, s, qkv, gq, bq, gk, bk, ws, ws_bytes);
+  if (rc) return rc;
+  if ((rc = check_core_args(mode, s, qkv, attn, ws, ws_bytes))) return rc;
+  if (!x || !w_qkv || !w_out || !y) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(w_qkv, 16) || !aligned(w_out, 16) || !aligned(y, 16) ||
+      (b_qkv && !aligned(b_qkv, 16)) || (b_out && !aligned(b_out, 16)))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  const long long M = static_cast<long long>(s->S) * s->T, C = static_cast<long long>(s->H) * 64;
+  if ((rc = check_linear_dims(M, 3 * C, C))) return rc;
+  if (mode == VGGT_ATTN_REGISTER && 3LL * s->n_special > s->T) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  const size_t row = static_cast<size_t>(C) * 2;
+  const size_t x_bytes = M * row, qkv_bytes = 3 * M * row;
+  if (overlaps(y, x_bytes, attn, x_bytes) || overlaps(y, x_bytes, ws, ws_bytes) || overlaps(y, x_bytes, qkv, qkv_bytes) ||
+      overlaps(y, x_bytes, x, x_bytes) || overlaps(qkv, qkv_bytes, x, x_bytes) || overlaps(attn, x_bytes, x, x_bytes) ||
+      overlaps(ws, ws_bytes, x, x_bytes))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+}  // namespace
+
 extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const void* x, const void* w_qkv,
                                const float* b_qkv, const float* q_gamma, const float* q_beta, const float* k_gamma,
                                const float* k_beta, const void* w_out, const float* b_out, void* qkv, void* attn,
                                void* y, void* workspace, size_t workspace_bytes, void* cuda_stream) {
-  int rc = check_qkv_proj_args(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, workspace,
-                               workspace_bytes);
+  int rc = check_block_args(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, w_out, b_out, qkv, attn, y,
+                            workspace, workspace_bytes);
   if (rc) return rc;
-  if ((rc = check_core_args(mode, shape, qkv, attn, workspace, workspace_bytes))) return rc;
-  const long long M = static_cast<long long>(shape->S) * shape->T, C = static_cast<long long>(shape->H) * 64;
-  if (!w_out || !y) return VGGT_ATTN_ERR_INVALID_ARG;
-  if (!aligned(w_out, 16) || !aligned(y, 16) || (b_out && !aligned(b_out, 16))) return VGGT_ATTN_ERR_MISALIGNED;
-  const size_t y_bytes = static_cast<size_t>(M) * C * 2;
-  if (overlaps(y, y_bytes, attn, y_bytes) || overlaps(y, y_bytes, workspace, workspace_bytes) ||
-      overlaps(y, y_bytes, qkv, static_cast<size_t>(M) * 3 * C * 2) || overlaps(y, y_bytes, x, y_bytes))
-    return VGGT_ATTN_ERR_INVALID_ARG;
   if ((rc = check_device())) return rc;
+  const long long M = static_cast<long long>(shape->S) * shape->T, C = static_cast<long long>(shape->H) * 64;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  if (mode == VGGT_ATTN_REGISTER) {
+    // Only the special tokens take part: gather their rows of x, run the block
+    // on that compact sequence (register attention over it is global attention
+    // without rotation), scatter the result rows back; patch rows of y are not
+    // written.  Scratch: attn holds x_s, attn_s and y_s; qkv holds qkv_s.
+    vggt_attn_shape s2 = *shape;
+    s2.T = shape->n_special;
+    s2.grid_h = 0;
+    s2.grid_w = 0;
+    const long long Ms = static_cast<long long>(shape->S) * shape->n_special;
+    const size_t row = static_cast<size_t>(C) * 2;
+    uint8_t* xs = static_cast<uint8_t*>(attn);
+    uint8_t* as = xs + Ms * row;
+    uint8_t* ys = as + Ms * row;
+    const WorkspaceView wv = workspace_view(&s2, VGGT_ATTN_GLOBAL, workspace);
+    if ((rc = launch_special_rows(x, xs, static_cast<int>(Ms), row, shape->n_special, shape->T, true, st))) return rc;
+    if ((rc = launch_linear_plain(xs, w_qkv, b_qkv, qkv, Ms, 3 * C, C, wv.status, st))) return rc;
+    if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, &s2, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st))) return rc;
+    if ((rc = launch_core(VGGT_ATTN_GLOBAL, &s2, qkv, as, wv, st))) return rc;
+    if ((rc = launch_linear_plain(as, w_out, b_out, ys, Ms, C, C, wv.status, st))) return rc;
+    return launch_special_rows(ys, y, static_cast<int>(Ms), row, shape->n_special, shape->T, false, st);
+  }
   const WorkspaceView wv = workspace_view(shape, mode, workspace);
   // QKV projection as a plain GEMM into qkv, then the prologue: measured
   // faster than the fused projection (whose LayerNorm/RoPE epilogue, not its
   // products, sets its time) on both the frame and the global workloads.
-  {
-    vggt::LinearParams pq{};
-    pq.M = static_cast<int>(M);
-    pq.N = static_cast<int>(3 * C);
-    pq.K = static_cast<int>(C);
-    pq.bias = b_qkv;
-    pq.status = wv.status;
-    pq.grid_w = 1;
-    CUtensorMap mqkv;
-    if (!make_rows_map(&mqkv, qkv, 3 * C, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
-    if ((rc = launch_linear(pq, x, w_qkv, mqkv, mqkv, mqkv, 0, 0, st))) return rc;
-  }
+  if ((rc = launch_linear_plain(x, w_qkv, b_qkv, qkv, M, 3 * C, C, wv.status, st))) return rc;
   if ((rc = launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st))) return rc;
   if ((rc = launch_core(mode, shape, qkv, attn, wv, st))) return rc;
-  vggt::LinearParams p{};
-  p.M = static_cast<int>(M);
-  p.N = static_cast<int>(C);
-  p.K = static_cast<int>(C);
-  p.bias = b_out;
-  p.status = wv.status;
-  p.grid_w = 1;
-  CUtensorMap my;
-  if (!make_rows_map(&my, y, C, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
-  return launch_linear(p, attn, w_out, my, my, my, 0, 0, st);
+  return launch_linear_plain(attn, w_out, b_out, y, M, C, C, wv.status, st);
 }
 
 // ---------------------------------------------------------------------------
