@@ -66,6 +66,22 @@ def test_constant_v_gives_constant_output():
     assert np.abs(got - want[None]).max() <= 2 ** -7 * np.abs(want).max()
 
 
+# Frame mode runs persistent CTAs (two per SM) that each take several (tile, head, frame) units in turn;
+# these shapes have more units than the grid has CTAs, with one key step per unit (T <= 64), a single
+# ragged tile per unit, and a second tile holding only 2 rows.
+MANY_UNITS = [
+    shp(700, 1, 5, 4, 4),        # T = 21: 700 units of one key step
+    shp(400, 2, 17, 7, 13),      # T = 108: 800 units of one ragged tile, two key steps
+    shp(300, 1, 2, 8, 16),       # T = 130: 600 units, every second one with 2 valid rows
+]
+
+
+@pytest.mark.parametrize("shape", MANY_UNITS, ids=[f"S{s.S}T{s.T}H{s.H}" for s in MANY_UNITS])
+def test_frame_more_units_than_ctas(shape):
+    x = W.make_random_inputs(shape, 300 + shape.T)
+    check_mode("frame", shape, x)
+
+
 # ------------------------------------------------------------------ the workloads at full size (sampled)
 def test_workload1_frame_full():
     w = W.workload(1)

@@ -17,7 +17,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libvggt_attn.so")
 SOURCES = [os.path.join(HERE, "csrc", "vggt_attn.cu")]
 DEPENDS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
-                     ("attention_sm100.cuh", "linear_sm100.cuh", "prologue.cuh", "sga.cuh", "common.cuh", "ptx_sm100.cuh")] + \
+                     ("attention_sm100.cuh", "attention_frame_persistent.cuh", "linear_sm100.cuh", "prologue.cuh", "sga.cuh", "common.cuh", "ptx_sm100.cuh")] + \
           [os.path.join(ROOT, "include", "vggt_attn.h")]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -1,0 +1,450 @@
+// Frame-mode attention core with persistent CTAs (VGGT-Omega Aggregator
+// explainer, section 3, step 1: each frame's tokens attend within the frame).
+//
+// A frame problem has only ceil(T/64) = 17 key steps per 128-query tile, so a
+// CTA that computes one tile spends a large share of its life starting up
+// (barrier set-up, TMEM allocation, first loads from HBM) and draining.  Here
+// each CTA (two per SM, 256 threads, 256 TMEM columns) walks the units
+// u = blockIdx.x, blockIdx.x + gridDim.x, ... (unit = one 128-query tile of
+// one (frame, head), tiles of a problem consecutive) and keeps its pipeline
+// running across units: the producer loads the next unit's Q into a second
+// buffer and its K/V into the same ring, the softmax warps copy the next Q
+// into TMEM as soon as the current unit's last QK^T product has completed,
+// so the next unit's first products run during this unit's epilogue.  The
+// per-step work is that of attn_core_kernel (see attention_sm100.cuh): Q in
+// TMEM, two S buffers, PV with 16 ones columns for the row sums, online
+// softmax with a lazily moved reference max.  Barrier phases run on across
+// units.  Every wait is bounded.
+#pragma once
+
+#include <cstdint>
+
+#include "attention_sm100.cuh"
+
+namespace vggt {
+
+namespace fp {
+using core::BM;
+using core::BN;
+using core::D;
+using core::KV_BYTES;
+using core::Q_BYTES;
+constexpr int STAGES = 4;
+constexpr int OFF_Q = 0;                                // two Q buffers
+constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
+constexpr int OFF_ONES = OFF_V + STAGES * KV_BYTES;
+constexpr int OFF_BAR = OFF_ONES + KV_BYTES;
+enum {
+  BAR_Q_FULL = 0,                       // [Q buffer]
+  BAR_Q_EMPTY = BAR_Q_FULL + 2,         // [Q buffer]
+  BAR_KV_FULL = BAR_Q_EMPTY + 2,
+  BAR_KV_EMPTY = BAR_KV_FULL + STAGES,
+  BAR_S_FULL = BAR_KV_EMPTY + STAGES,   // [buffer]
+  BAR_P_FULL = BAR_S_FULL + 2,          // [buffer]
+  BAR_PV_DONE = BAR_P_FULL + 2,
+  BAR_O_FINAL = BAR_PV_DONE + 1,
+  BAR_O_FREE = BAR_O_FINAL + 1,         // O read out by the epilogue
+  BAR_Q_TMEM = BAR_O_FREE + 1,          // Q copied into TMEM
+  BAR_DRAIN = BAR_Q_TMEM + 1,
+  N_BARS = BAR_DRAIN + 1
+};
+constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;          // tmem slot, abort flag
+constexpr int SMEM_BYTES = OFF_MISC + 16;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+constexpr int THREADS = 256;
+constexpr int CTAS_PER_SM = 2;
+constexpr uint32_t TMEM_COLS = 256;
+constexpr uint32_t COL_O = 128;                         // S buffers at 0 and 64
+constexpr uint32_t COL_Q = COL_O + core::NV;
+constexpr int REGS_AT_LAUNCH = 128;
+constexpr int REGS_PRODUCER = 56;
+constexpr int REGS_SOFTMAX = 200;
+static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 128 <= REGS_AT_LAUNCH * THREADS, "register split too large");
+static_assert(SMEM_ALLOC * CTAS_PER_SM <= 227 * 1024, "two CTAs per SM");
+}  // namespace fp
+
+struct FrameUnits {
+  int n_qt;       // 128-query tiles per (frame, head)
+  int n_units;    // n_qt * H * S
+};
+
+__device__ __forceinline__ void frame_unit(const CoreParams& p, const FrameUnits& fu, int u, int& q0, int& h, int& b) {
+  const int qt = u % fu.n_qt;
+  const int r = u / fu.n_qt;
+  h = r % p.H;
+  b = r / p.H;
+  q0 = qt * fp::BM;
+}
+
+__device__ __forceinline__ void mbar_arrive_count(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+// Softmax warpgroup (warps 4-7): thread r owns query row r of every unit.
+__device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const FrameUnits& fu, const uint8_t* smem,
+                                                   uint32_t tmem, uint32_t bar0, volatile int* abort_flag, int n_kv,
+                                                   int warp, int lane) {
+  using namespace fp;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  const int quarter = warp & 3;
+  const int row = quarter * 32 + lane;
+  const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
+  const uint32_t s_base = tmem + lane_base;
+  const uint32_t o_addr = tmem + lane_base + COL_O;
+  const PolyConsts pc = poly_consts();
+  const bool leader = (threadIdx.x & 127) == 0;
+
+  // Q tile of local unit i (buffer i % 2, 128-byte swizzle) -> TMEM columns
+  // COL_Q.. (row r in lane r, dims (2c, 2c+1) in column c).
+  auto copy_q = [&](int i) -> bool {
+    bool ok = wait_bounded(bar(BAR_Q_FULL + (i & 1)), (i >> 1) & 1, abort_flag, p.status, p.timeout_ns, 0x630u);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) return false;
+    const uint4* qrow = reinterpret_cast<const uint4*>(smem + OFF_Q + (i & 1) * Q_BYTES + row * 128);
+    uint32_t qr[32];
+#pragma unroll
+    for (int c = 0; c < 8; ++c) {
+      const uint4 v = qrow[c ^ (row & 7)];
+      qr[4 * c] = v.x;
+      qr[4 * c + 1] = v.y;
+      qr[4 * c + 2] = v.z;
+      qr[4 * c + 3] = v.w;
+    }
+    tmem_st32(tmem + lane_base + COL_Q, qr);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar(BAR_Q_TMEM));
+    mbar_arrive(bar(BAR_Q_EMPTY + (i & 1)));
+    return true;
+  };
+
+  bool ok = true;
+  bool q_ready = false;
+  int G = 0;                                    // key steps done by this CTA
+  const int c_pv = n_kv < 2 ? n_kv : 2;         // PV_DONE commits per unit
+  for (int i = 0;; ++i) {
+    const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+    if (u >= fu.n_units) break;
+    int q0, h, b;
+    frame_unit(p, fu, u, q0, h, b);
+    if (!q_ready) {
+      ok = copy_q(i);
+      if (!ok) break;
+    }
+    q_ready = false;
+    const int kv0 = i * n_kv;
+    float m_run = -INFINITY;
+    for (int j = 0; j < n_kv; ++j) {
+      const int g = G + j;
+      const int buf = g & 1;
+      const uint32_t s_addr = s_base + buf * BN;
+      ok = wait_bounded(bar(BAR_S_FULL + buf), (g >> 1) & 1, abort_flag, p.status, p.timeout_ns, 0x600u);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      // S(j) complete => PV(j-2) complete: its K/V stage is free.
+      if (j >= 2 && leader) mbar_arrive(bar(BAR_KV_EMPTY + (kv0 + j - 2) % STAGES));
+      tc_fence_after();
+      uint32_t sr[2][32];
+      tmem_ld32(s_addr, sr[0]);
+      tmem_ld32(s_addr + 32, sr[1]);
+      tmem_wait_ld();
+      const int valid = p.Lk - j * BN;
+      if (valid < BN) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e >= valid) sr[c][e] = __float_as_uint(-INFINITY);
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < 32; e += 2) {
+        mx0 = max3f(mx0, __uint_as_float(sr[0][e]), __uint_as_float(sr[0][e + 1]));
+        mx1 = max3f(mx1, __uint_as_float(sr[1][e]), __uint_as_float(sr[1][e + 1]));
+      }
+      const float tile_max = fmaxf(mx0, mx1);
+      const bool move = (j == 0) || (tile_max > m_run + core::RESCALE_THRESHOLD);
+      float alpha = 1.f;
+      if (move) {
+        alpha = (j == 0) ? 0.f : ex2_approx(m_run - tile_max);
+        m_run = tile_max;
+      }
+      const float neg_m = -m_run;
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float x0, x1, p0, p1;
+          add_x2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]), neg_m, neg_m, x0, x1);
+          const int pair = (c * 32 + e) >> 1;
+          if ((core::POLY_PAIR_MASK >> (pair & 7)) & 1u) {
+            exp2_poly_x2(x0, x1, p0, p1, pc);
+          } else {
+            p0 = ex2_approx(x0);
+            p1 = ex2_approx(x1);
+          }
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tmem_st16(s_addr + c * 16, pk);
+      }
+      // Rescale O after PV(j-1) (S(j+1) was issued after it; past the unit's
+      // last S, the unit's first PV_DONE commit says so).
+      if (__any_sync(0xffffffffu, move && j > 0)) {
+        ok = (j + 1 < n_kv) ? wait_bounded(bar(BAR_S_FULL + ((g + 1) & 1)), ((g + 1) >> 1) & 1, abort_flag, p.status,
+                                           p.timeout_ns, 0x610u)
+                            : wait_bounded(bar(BAR_PV_DONE), (i * c_pv) & 1, abort_flag, p.status, p.timeout_ns,
+                                           0x618u);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t orr[2][32], osum;
+        tmem_ld32(o_addr, orr[0]);
+        tmem_ld32(o_addr + 32, orr[1]);
+        tmem_ld1(o_addr + D, osum);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[c][e] = __float_as_uint(__uint_as_float(orr[c][e]) * alpha);
+        osum = __float_as_uint(__uint_as_float(osum) * alpha);
+        tmem_st32(o_addr, orr[0]);
+        tmem_st32(o_addr + 32, orr[1]);
+        tmem_st1(o_addr + D, osum);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(BAR_P_FULL + buf));
+    }
+    if (!ok) break;
+    // Next unit's Q into TMEM now (every QK^T product of this unit is done),
+    // so that its first products run during this epilogue.
+    if (u + static_cast<int>(gridDim.x) < fu.n_units) {
+      ok = copy_q(i + 1);
+      if (!ok) break;
+      q_ready = true;
+    }
+    ok = wait_bounded(bar(BAR_O_FINAL), i & 1, abort_flag, p.status, p.timeout_ns, 0x620u);
+    ok = __all_sync(0xffffffffu, ok);
+    if (!ok) break;
+    tc_fence_after();
+    if (leader)
+      for (int j = n_kv > 2 ? n_kv - 2 : 0; j < n_kv; ++j) mbar_arrive(bar(BAR_KV_EMPTY + (kv0 + j) % STAGES));
+    uint32_t orr[2][32], osum;
+    tmem_ld32(o_addr, orr[0]);
+    tmem_ld32(o_addr + 32, orr[1]);
+    tmem_ld1(o_addr + D, osum);
+    tmem_wait_ld();
+    tc_fence_before();
+    mbar_arrive(bar(BAR_O_FREE));
+    const int qi = q0 + row;
+    if (qi < p.L) {
+      const float inv = 1.f / __uint_as_float(osum);
+      const long long out_row = static_cast<long long>(b) * p.out_T +
+                                static_cast<long long>(qi / p.out_group) * p.out_T + (qi % p.out_group);
+      uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D);
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+          uint4 w;
+          const uint32_t* o = &orr[c][v * 8];
+          w.x = pack_bf16x2(__uint_as_float(o[0]) * inv, __uint_as_float(o[1]) * inv);
+          w.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
+          w.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
+          w.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
+          dst[c * 4 + v] = w;
+        }
+      }
+    }
+    G += n_kv;
+  }
+}
+
+// Grid: min(n_units, 2 x SMs) CTAs, one dimension.  The producer runs ahead
+// of the softmax by up to one unit of Q and STAGES key steps of K/V.
+__global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
+    attn_frame_persistent_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                                 const __grid_constant__ CUtensorMap tmap_v, const CoreParams p,
+                                 const FrameUnits fu) {
+  using namespace fp;
+  using core::IDESC_PV;
+  using core::IDESC_QK;
+  using core::NV;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
+  volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n_kv = (p.Lk + BN - 1) / BN;
+
+  if (threadIdx.x == 0) {
+    for (int qb = 0; qb < 2; ++qb) {
+      mbar_init(bar(BAR_Q_FULL + qb), 1);
+      mbar_init(bar(BAR_Q_EMPTY + qb), 128);
+    }
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar(BAR_KV_FULL + s), 1);
+      mbar_init(bar(BAR_KV_EMPTY + s), 1);
+    }
+    for (int buf = 0; buf < 2; ++buf) {
+      mbar_init(bar(BAR_S_FULL + buf), 1);
+      mbar_init(bar(BAR_P_FULL + buf), 128);
+    }
+    mbar_init(bar(BAR_PV_DONE), 1);
+    mbar_init(bar(BAR_O_FINAL), 1);
+    mbar_init(bar(BAR_O_FREE), 128);
+    mbar_init(bar(BAR_Q_TMEM), 128);
+    mbar_init(bar(BAR_DRAIN), 1);
+    fence_mbar_init();
+    *abort_flag = status_is_set(p.status) ? 1 : 0;  // another CTA already failed: skip the work
+    tma_prefetch_desc(&tmap_q);
+    tma_prefetch_desc(&tmap_k);
+    tma_prefetch_desc(&tmap_v);
+  }
+  for (int e = threadIdx.x; e < KV_BYTES / 16; e += blockDim.x)
+    reinterpret_cast<uint4*>(smem + OFF_ONES)[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  if (warp == 1) {
+    tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const bool skip = *abort_flag != 0;
+
+  if (warp >= 4) {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
+    if (!skip) frame_softmax_role(p, fu, smem, tmem, bar0, abort_flag, n_kv, warp, lane);
+  } else {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
+  }
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && !skip) {
+      int kv_issued[STAGES];
+      for (int s = 0; s < STAGES; ++s) kv_issued[s] = 0;
+      int q_issued[2] = {0, 0};
+      bool ok = true;
+      for (int i = 0; ok; ++i) {
+        const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+        if (u >= fu.n_units) break;
+        int q0, h, b;
+        frame_unit(p, fu, u, q0, h, b);
+        const int qb = i & 1;
+        if (i >= 2) {
+          ok = wait_bounded(bar(BAR_Q_EMPTY + qb), ((i >> 1) - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x580u);
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(bar(BAR_Q_FULL + qb), Q_BYTES);
+        tma_load_3d(sbase + OFF_Q + qb * Q_BYTES, &tmap_q, bar(BAR_Q_FULL + qb), 0, q0, h * p.B + b);
+        ++q_issued[qb];
+        for (int j = 0; j < n_kv; ++j) {
+          const int k = i * n_kv + j;
+          const int st = k % STAGES;
+          if (k >= STAGES) {
+            ok = wait_bounded(bar(BAR_KV_EMPTY + st), ((k / STAGES) - 1) & 1, abort_flag, p.status, p.timeout_ns,
+                              0x500u | st);
+            if (!ok) break;
+          }
+          mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * KV_BYTES);
+          tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
+          tma_load_4d(sbase + OFF_V + st * KV_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+          ++kv_issued[st];
+        }
+      }
+      if (!ok) {
+        // Drain: the last load issued into every stage and Q buffer must land
+        // before this CTA's shared memory is released.
+        for (int qb = 0; qb < 2; ++qb)
+          if (q_issued[qb] > 0) wait_drain(bar(BAR_Q_FULL + qb), (q_issued[qb] - 1) & 1, p.timeout_ns);
+        for (int st = 0; st < STAGES; ++st)
+          if (kv_issued[st] > 0) wait_drain(bar(BAR_KV_FULL + st), (kv_issued[st] - 1) & 1, p.timeout_ns);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && !skip) {
+      const uint64_t dk = smem_desc_sw128(sbase + OFF_K, 16, 1024);
+      const uint32_t t_o = tmem + COL_O, t_q = tmem + COL_Q;
+      auto issue_s = [&](int g, int k) {   // S of step g into buffer g % 2, K from load k, Q from TMEM
+        const uint64_t kd = dk + (k % STAGES) * (KV_BYTES >> 4);
+        const uint32_t d = tmem + (g & 1) * BN;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) mma_ts(d, t_q + kk * 8, kd + 2 * kk, IDESC_QK, kk > 0);
+      };
+      auto issue_pv = [&](int g, int k, bool first) {   // O (+)= P(g) [V(k) | 1]
+        const uint32_t v_addr = sbase + OFF_V + (k % STAGES) * KV_BYTES;
+        const uint64_t v = smem_desc_sw128(v_addr, sbase + OFF_ONES - v_addr, 1024);
+        const uint32_t a = tmem + (g & 1) * BN;
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(t_o, a + kk * 8, v + kk * (2048 >> 4), IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+      };
+      bool ok = true;
+      int G = 0;
+      for (int i = 0; ok; ++i) {
+        const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
+        if (u >= fu.n_units) break;
+        const int kv0 = i * n_kv;
+        ok = wait_bounded(bar(BAR_Q_TMEM), i & 1, abort_flag, p.status, p.timeout_ns, 0x540u);
+        for (int jj = 0; jj < 2 && jj < n_kv && ok; ++jj) {
+          const int k = kv0 + jj;
+          ok = wait_bounded(bar(BAR_KV_FULL + k % STAGES), (k / STAGES) & 1, abort_flag, p.status, p.timeout_ns,
+                            0x510u | jj);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(G + jj, k);
+          tc_commit(bar(BAR_S_FULL + ((G + jj) & 1)));
+        }
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int g = G + j;
+          const int jn = j + 2;
+          if (jn < n_kv) {   // K/V of step j+2 first (normally long resident)
+            const int kn = kv0 + jn;
+            ok = wait_bounded(bar(BAR_KV_FULL + kn % STAGES), (kn / STAGES) & 1, abort_flag, p.status,
+                              p.timeout_ns, 0x530u);
+            if (!ok) break;
+          }
+          ok = wait_bounded(bar(BAR_P_FULL + (g & 1)), (g >> 1) & 1, abort_flag, p.status, p.timeout_ns, 0x520u);
+          if (!ok) break;
+          if (j == 0 && i > 0) {   // the previous unit's epilogue has read O
+            ok = wait_bounded(bar(BAR_O_FREE), (i - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
+            if (!ok) break;
+          }
+          tc_fence_after();
+          issue_pv(g, kv0 + j, j == 0);
+          if (jn < n_kv) {
+            issue_s(g + 2, kv0 + jn);
+            tc_commit(bar(BAR_S_FULL + (g & 1)));   // also covers PV(j)
+          } else {
+            tc_commit(bar(BAR_PV_DONE));
+            if (j == n_kv - 1) tc_commit(bar(BAR_O_FINAL));
+          }
+        }
+        G += n_kv;
+      }
+      if (!ok) {  // let every MMA already issued finish before TMEM is released
+        tc_commit(bar(BAR_DRAIN));
+        wait_drain(bar(BAR_DRAIN), 0, p.timeout_ns);
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, TMEM_COLS);
+  }
+}
+
+}  // namespace vggt

@@ -109,9 +109,11 @@ constexpr uint32_t POLY_PAIR_MASK = 0x80u;
 
 // Per-CTA shape of the kernel.  NQ = 2: two 128-query tiles share every K/V
 // tile (one CTA per SM; global and register mode, whose key loops are long).
-// NQ = 1: one tile per CTA and two CTAs per SM (frame mode: 17 key steps per
-// tile, so a CTA's start and end are a large share of its life, and the other
-// CTA on the SM keeps the tensor core and the MUFU unit busy meanwhile).
+// NQ = 1: one tile per CTA and two CTAs per SM, one launch-time CTA per tile.
+// Frame mode (17 key steps per tile) runs the persistent form of the NQ = 1
+// shape instead (attention_frame_persistent.cuh): its CTAs take tile after
+// tile and start the next tile's products during the last one's epilogue,
+// 2 % faster on the 500-frame workload.
 template <int NQ_, bool SGA_ = false>
 struct CoreCfg {
   static constexpr int NQ = NQ_;

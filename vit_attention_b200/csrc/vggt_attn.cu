@@ -10,6 +10,7 @@
 #include <cstring>
 #include <mutex>
 
+#include "attention_frame_persistent.cuh"
 #include "attention_sm100.cuh"
 #include "linear_sm100.cuh"
 #include "prologue.cuh"
@@ -204,6 +205,33 @@ int launch_core_cfg(const ModeGeometry& g, int H, const CUtensorMap& mq, const C
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
+// Frame mode: persistent CTAs, two per SM, each walking the (tile, head,
+// frame) units with a stride of the grid size.
+int launch_frame_persistent(const ModeGeometry& g, int H, const CUtensorMap& mq, const CUtensorMap& mk,
+                            const CUtensorMap& mv, const vggt::CoreParams& p, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(vggt::attn_frame_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           vggt::fp::SMEM_ALLOC) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  cudaFuncAttributes fa;   // the register split assumes the compiled count (see launch_core_cfg)
+  if (cudaFuncGetAttributes(&fa, vggt::attn_frame_persistent_kernel) != cudaSuccess ||
+      fa.numRegs < vggt::fp::REGS_AT_LAUNCH)
+    return VGGT_ATTN_ERR_CUDA;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  vggt::FrameUnits fu;
+  fu.n_qt = static_cast<int>((g.L + vggt::core::BM - 1) / vggt::core::BM);
+  const long long n_units = static_cast<long long>(fu.n_qt) * H * g.B;
+  if (n_units > INT32_MAX) return VGGT_ATTN_ERR_INVALID_ARG;
+  fu.n_units = static_cast<int>(n_units);
+  long long grid = static_cast<long long>(sms) * vggt::fp::CTAS_PER_SM;
+  if (grid > n_units) grid = n_units;
+  vggt::attn_frame_persistent_kernel<<<static_cast<unsigned>(grid), vggt::fp::THREADS, vggt::fp::SMEM_ALLOC,
+                                       stream>>>(mq, mk, mv, p, fu);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
 int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, const WorkspaceView& w,
                 cudaStream_t stream) {
   const ModeGeometry g = geometry(s, mode);
@@ -244,7 +272,7 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   p.timeout_ns = kDefaultTimeoutNs;
   // Frame mode: one query tile per CTA, two CTAs per SM; global and register
   // mode: two query tiles per CTA sharing every K/V tile.
-  if (mode == VGGT_ATTN_FRAME) return launch_core_cfg<vggt::CoreCfg<1>>(g, s->H, mq, mk, mv, p, stream);
+  if (mode == VGGT_ATTN_FRAME) return launch_frame_persistent(g, s->H, mq, mk, mv, p, stream);
   return launch_core_cfg<vggt::CoreCfg<2>>(g, s->H, mq, mk, mv, p, stream);
 }
 
