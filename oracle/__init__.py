@@ -51,3 +51,11 @@ from .attention import (  # noqa: F401
 )
 from .projection import attention_block, linear, projected_qkv  # noqa: F401
 from .sga import attn_global_sga, sga_kept_tokens  # noqa: F401
+from .block import (  # noqa: F401
+    N_LAYERS,
+    REGISTER_LAYERS,
+    aggregator_forward,
+    block_forward,
+    gelu,
+    token_layer_norm,
+)

@@ -57,7 +57,8 @@ def patch_row_col(t: np.ndarray, n_special: int, grid_w: int) -> Tuple[np.ndarra
     t = np.asarray(t, dtype=np.int64)
     is_patch = t >= n_special
     p = np.where(is_patch, t - n_special, 0)
-    return is_patch, p // grid_w, p % grid_w
+    gw = grid_w if grid_w > 0 else 1          # a frame of special tokens only has no patch grid
+    return is_patch, p // gw, p % gw
 
 
 def _rotate_half_block(x: np.ndarray, pos: np.ndarray, omega: np.ndarray) -> np.ndarray:

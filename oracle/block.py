@@ -1,0 +1,88 @@
+"""fp64 oracle of the transformer blocks and the alternating-attention layer
+schedule around the attention core (test infrastructure).
+
+Source, cited by page title and section:
+  [P1] VGGT-Omega Aggregator explainer -- section 3: the Aggregator is 24
+       layers deep; every layer runs a frame block (attention within each
+       frame, with 2D RoPE) and then an inter-frame block, global (all tokens
+       of all frames) except at the layer indices [2, 6, 9, 14, 20], where
+       only the 17 camera + register tokens of every frame take part and the
+       patch tokens stay in their own frame's path; the attention layers use
+       Q/K normalisation together with LayerScale (initial value 1e-5).
+  [P1] section 2: the patch tokens come from a DINO-style ViT, whose block
+       the Aggregator's blocks follow.
+
+Readings where the page is silent (listed in the design doc):
+  * A block is the pre-norm transformer block of a DINO-style ViT:
+        x <- x + ls1 * proj(attention(qkv(norm1(x))))
+        x <- x + ls2 * fc2(GELU(fc1(norm2(x))))
+    norm1/norm2 are LayerNorms over the C channels of a token (biased
+    variance, caller-given epsilon); the MLP hidden width is 4C; GELU is the
+    exact form x * Phi(x); ls1, ls2 are per-channel LayerScale vectors.
+  * In a register layer the whole inter-frame block (both residual branches)
+    acts on the special tokens only; patch tokens pass through unchanged.
+  * The attention inside a block is the core's (QK-LayerNorm, RoPE on patch
+    tokens, softmax attention in the block's mode) on the block's own qkv.
+"""
+from __future__ import annotations
+
+import numpy as np
+from scipy.special import erf
+
+from .attention import HEAD_DIM, attn_mode, bf16_to_f64, register_tokens
+
+REGISTER_LAYERS = (2, 6, 9, 14, 20)      # [P1] section 3
+N_LAYERS = 24                            # [P1] section 3
+
+
+def token_layer_norm(x: np.ndarray, gamma, beta, eps: float) -> np.ndarray:
+    """LayerNorm over the last axis (the C channels of a token), biased variance."""
+    mu = x.mean(axis=-1, keepdims=True)
+    var = ((x - mu) ** 2).mean(axis=-1, keepdims=True)
+    return (x - mu) / np.sqrt(var + eps) * np.asarray(gamma, np.float64) + np.asarray(beta, np.float64)
+
+
+def gelu(x: np.ndarray) -> np.ndarray:
+    """x * Phi(x), Phi the standard normal distribution function."""
+    return x * 0.5 * (1.0 + erf(x / np.sqrt(2.0)))
+
+
+def _affine(x: np.ndarray, w_bits, b) -> np.ndarray:
+    y = x @ bf16_to_f64(w_bits).T
+    return y if b is None else y + np.asarray(b, np.float64)
+
+
+def block_forward(mode: str, shape, x, w, norm_eps: float) -> np.ndarray:
+    """One block applied to token features x (bf16 bits or fp64, ``[S*T, C]``).
+
+    Returns fp64 ``[S*T, C]``.  mode: "frame", "global" or "register"; in
+    register mode only the rows of the special tokens change.
+    """
+    x = bf16_to_f64(x) if x.dtype == np.uint16 else np.asarray(x, np.float64)
+    C = shape.H * HEAD_DIM
+    rows = register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T, dtype=np.int64)
+    # Attention branch: qkv of every token (only rows in `rows` are read in
+    # register mode, whose keys and queries are the special tokens).
+    h = token_layer_norm(x, w["norm1_gamma"], w["norm1_beta"], norm_eps)
+    qkv = _affine(h, w["w_qkv"], w.get("b_qkv")).reshape(shape.S, shape.T, 3, shape.H, HEAD_DIM)
+    inputs = {"qkv_f64": qkv}
+    for name in ("q_gamma", "q_beta", "k_gamma", "k_beta"):
+        inputs[name] = w[name]
+    a = attn_mode(mode, shape, inputs, rows).reshape(len(rows), C)
+    y = x.copy()
+    xr = x[rows] + np.asarray(w["ls1"], np.float64) * _affine(a, w["w_proj"], w.get("b_proj"))
+    # MLP branch on the same rows.
+    h2 = token_layer_norm(xr, w["norm2_gamma"], w["norm2_beta"], norm_eps)
+    u = gelu(_affine(h2, w["w_fc1"], w.get("b_fc1")))
+    y[rows] = xr + np.asarray(w["ls2"], np.float64) * _affine(u, w["w_fc2"], w.get("b_fc2"))
+    return y
+
+
+def aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, norm_eps: float) -> np.ndarray:
+    """Layer l: the frame block frame_blocks[l], then the inter-frame block
+    inter_blocks[l], in register mode if l is in register_layers, else global."""
+    y = bf16_to_f64(x) if x.dtype == np.uint16 else np.asarray(x, np.float64)
+    for l, (fw, iw) in enumerate(zip(frame_blocks, inter_blocks)):
+        y = block_forward("frame", shape, y, fw, norm_eps)
+        y = block_forward("register" if l in register_layers else "global", shape, y, iw, norm_eps)
+    return y

@@ -186,6 +186,51 @@ def make_block_inputs(shape: Shape, seed: int) -> Dict[str, np.ndarray]:
     return out
 
 
+def make_tokens(shape: Shape, seed: int) -> np.ndarray:
+    """Seeded token features x: bf16 bits ``[S*T, C]`` ~ N(0, 1), frame s from ``default_rng([seed, 4, s])``."""
+    S, T, C = shape.S, shape.T, shape.H * shape.head_dim
+    x = np.empty((S * T, C), dtype=np.uint16)
+    for s in range(S):
+        x[s * T:(s + 1) * T] = f32_to_bf16_bits(
+            np.random.default_rng([seed, 4, s]).standard_normal((T, C), dtype=np.float32))
+    return x
+
+
+def make_transformer_block_weights(H: int, seed: int, head_dim: int = HEAD_DIM) -> Dict[str, np.ndarray]:
+    """Seeded weights of one pre-norm transformer block, C = H * head_dim, hidden width 4C.
+
+    Matrices are bf16 bits in nn.Linear layout ``[out][in]`` ~ N(0, 1/in) (each
+    product then has unit variance): w_qkv ``[3C, C]``, w_proj ``[C, C]``, w_fc1
+    ``[4C, C]``, w_fc2 ``[C, 4C]``.  Vectors are fp32: norm gammas and LayerScales
+    1 + 0.1 N(0, 1) (LayerScale drawn near 1, not at its 1e-5 initial value, so
+    that both branches of the block show in its output), norm betas and biases
+    0.1 N(0, 1); q/k gamma/beta as for the attention core.  Item k uses
+    ``default_rng([seed, 20 + k])``.
+    """
+    C = H * head_dim
+    out = make_norm_params(H, seed, head_dim)
+
+    def rng(k):
+        return np.random.default_rng([seed, 20 + k])
+
+    def mat(k, n_out, n_in):
+        sd = np.float32(1.0 / np.sqrt(n_in))
+        return f32_to_bf16_bits(rng(k).standard_normal((n_out, n_in), dtype=np.float32) * sd)
+
+    def vec(k, n, centre):
+        return (centre + 0.1 * rng(k).standard_normal(n)).astype(np.float32)
+
+    out["norm1_gamma"], out["norm1_beta"] = vec(0, C, 1.0), vec(1, C, 0.0)
+    out["w_qkv"], out["b_qkv"] = mat(2, 3 * C, C), vec(3, 3 * C, 0.0)
+    out["w_proj"], out["b_proj"] = mat(4, C, C), vec(5, C, 0.0)
+    out["ls1"] = vec(6, C, 1.0)
+    out["norm2_gamma"], out["norm2_beta"] = vec(7, C, 1.0), vec(8, C, 0.0)
+    out["w_fc1"], out["b_fc1"] = mat(9, 4 * C, C), vec(10, 4 * C, 0.0)
+    out["w_fc2"], out["b_fc2"] = mat(11, C, 4 * C), vec(12, C, 0.0)
+    out["ls2"] = vec(13, C, 1.0)
+    return out
+
+
 def query_subset(n_queries: int, count: int, seed: int) -> np.ndarray:
     """Sorted seeded subset of query indices (all of them if count >= n)."""
     if count >= n_queries:
