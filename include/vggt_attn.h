@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VGGT_ATTN_ABI_VERSION 2
+#define VGGT_ATTN_ABI_VERSION 3
 
 /* Return codes (0 = success). */
 enum {
@@ -259,6 +259,79 @@ int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s_w, const v
                          const float* q_gamma, const float* q_beta,
                          const float* k_gamma, const float* k_beta, void* out,
                          void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* ------------------------------------------------------------------------
+ * Transformer blocks and the alternating-attention layer schedule
+ * (VGGT-Omega Aggregator explainer, section 3: 24 layers, each a frame block
+ * followed by an inter-frame block, the inter-frame block global except at the
+ * register layers [2, 6, 9, 14, 20], where only the camera and register
+ * tokens take part; QK normalisation on and LayerScale in every attention
+ * block).  A block is the pre-norm transformer block of the backbone:
+ *
+ *   x <- x + ls1 * proj(attention(qkv(norm1(x))))
+ *   x <- x + ls2 * fc2(GELU(fc1(norm2(x))))
+ *
+ * norm1/norm2: LayerNorm over the C = 64 H channels of a token (biased
+ * variance, eps = norm_eps, fp32 arithmetic, bf16 result); qkv: [3C][C]
+ * weight, outputs ordered q | k | v, each [H][64]; attention: the mode's
+ * QK-LayerNorm, 2D RoPE and exact softmax attention of vggt_attn_frame /
+ * vggt_attn_global; proj: [C][C]; fc1: [4C][C] (hidden width 4C); GELU the
+ * exact erf form x * Phi(x); fc2: [C][4C]; ls1, ls2: per-channel LayerScale.
+ * Intermediates (norm outputs, qkv, attention output, hidden activations)
+ * are bf16; every GEMM accumulates in fp32 and its bias / GELU / LayerScale
+ * and residual add are applied in fp32 before the one bf16 rounding.
+ *
+ * Weights: all device pointers, caller-owned, bf16 matrices in nn.Linear
+ * layout [out][in], fp32 vectors; biases may be NULL (zero), every other
+ * pointer is required and 16-byte aligned. */
+typedef struct {
+  const float* norm1_gamma; const float* norm1_beta;   /* [C] */
+  const void* w_qkv; const float* b_qkv;               /* bf16 [3C][C], fp32 [3C] */
+  const float* q_gamma; const float* q_beta;           /* QK-LayerNorm of q, [H][64] */
+  const float* k_gamma; const float* k_beta;           /* QK-LayerNorm of k, [H][64] */
+  const void* w_proj; const float* b_proj;             /* bf16 [C][C], fp32 [C] */
+  const float* ls1;                                    /* [C] */
+  const float* norm2_gamma; const float* norm2_beta;   /* [C] */
+  const void* w_fc1; const float* b_fc1;               /* bf16 [4C][C], fp32 [4C] */
+  const void* w_fc2; const float* b_fc2;               /* bf16 [C][4C], fp32 [C] */
+  const float* ls2;                                    /* [C] */
+} vggt_block_weights;
+
+/* vggt_block_workspace_size: bytes of workspace vggt_block_forward needs for
+ * (shape, mode), or 0 if the shape or mode is invalid.  It covers the
+ * attention workspace and the bf16 intermediates (for register mode, of the
+ * S n_special special tokens only).
+ *
+ * vggt_block_forward: one block applied in place to x, bf16 [S][T][C]
+ * (C = 64 H, a multiple of 256, at most 2048).  Frame mode: attention within
+ * each frame; global mode: over all S T tokens.  Register mode: the block
+ * runs on the special tokens alone (their rows are gathered, go through the
+ * whole block with global attention among them, unrotated, and are scattered
+ * back); patch rows of x are left untouched.  Kernels: LayerNorm, QKV GEMM,
+ * attention prologue and core, projection GEMM with the LayerScale residual
+ * add in its epilogue, LayerNorm, fc1 GEMM with GELU in its epilogue, fc2 GEMM
+ * with the LayerScale residual add; the first kernel clears the workspace
+ * status word.  x must not overlap the workspace or any weight.
+ *
+ * vggt_aggregator_forward: n_layers layers applied in place to x; layer l runs
+ * vggt_block_forward(FRAME, frame_blocks[l]) and then the inter-frame block
+ * inter_blocks[l] in register mode if l is one of register_layers[0 ..
+ * n_register) and in global mode otherwise.  frame_blocks and inter_blocks
+ * are host arrays of n_layers weight sets; register_layers is a host array
+ * (NULL when n_register is 0).  The workspace must hold
+ * vggt_aggregator_workspace_size(shape) bytes, the larger of the frame and
+ * global (and register) block needs.
+ *
+ * All are asynchronous on cuda_stream, validate every argument before
+ * enqueueing anything and allocate nothing. */
+size_t vggt_block_workspace_size(const vggt_attn_shape* shape, int mode);
+int vggt_block_forward(int mode, const vggt_attn_shape* shape, void* x, const vggt_block_weights* w,
+                       float norm_eps, void* workspace, size_t workspace_bytes, void* cuda_stream);
+size_t vggt_aggregator_workspace_size(const vggt_attn_shape* shape);
+int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_block_weights* frame_blocks,
+                            const vggt_block_weights* inter_blocks, int n_layers, const int* register_layers,
+                            int n_register, float norm_eps, void* workspace, size_t workspace_bytes,
+                            void* cuda_stream);
 
 #ifdef __cplusplus
 }

@@ -14,8 +14,8 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 @pytest.fixture(scope="module")
 def V():
-    from vit_attention_b200 import build
-    build.build()
+    import __graft_entry__
+    __graft_entry__._build_module().build()
     import vit_attention_b200
     return vit_attention_b200
 
@@ -26,7 +26,7 @@ def declared_functions():
         if fn.endswith(".h"):
             text = open(os.path.join(ROOT, "include", fn)).read()
             text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
-            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(vggt_attn_\w+)\s*\(", text, flags=re.M)
+            names += re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(vggt_\w+)\s*\(", text, flags=re.M)
     return sorted(set(names))
 
 
@@ -36,7 +36,7 @@ def test_library_exports_every_declared_function(V):
     lib = ctypes.CDLL(V.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
-    assert V.vggt_attn_abi_version() == 2
+    assert V.vggt_attn_abi_version() == 3
 
 
 def test_error_strings(V):

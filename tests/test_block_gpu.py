@@ -1,0 +1,134 @@
+"""GPU parity of the transformer blocks and the alternating layer schedule
+(vggt_block_forward, vggt_aggregator_forward) against the fp64 oracle
+(oracle/block.py), through the C ABI binding.
+
+Tolerance.  The CUDA path stores the norm outputs, qkv, the attention output,
+the MLP hidden activations and the block output in bf16 (every GEMM
+accumulates in fp32).  The fp64 oracle with bf16 rounding at exactly those
+points gives, on these shapes, a relative Frobenius error of 2.8-3.1e-3 on the
+block output, 4.5-4.8e-3 on its update (output - input) and a largest
+element error of 1.9-2.8e-2 (outputs reach |y| ~ 6, where one bf16 ulp is
+3.1e-2).  The bounds below leave 2-3x room for the fp32 accumulation order
+and the attention core's own error: rel-Frobenius <= 1e-2 (output) and
+<= 1.5e-2 (update), max-abs <= 6e-2; twice that for four blocks in a row."""
+import numpy as np
+import pytest
+
+import oracle as O
+import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+EPS = 1e-6
+OUT_FRO, DELTA_FRO, MAX_ABS = 1e-2, 1.5e-2, 6e-2
+
+
+def shp(S, H, ns, gh, gw):
+    return W.Shape(S=S, T=ns + gh * gw, H=H, n_special=ns, grid_h=gh, grid_w=gw)
+
+
+def _dev_bits(a):
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def _dev_weights(w):
+    import torch
+    out = {}
+    for k, v in w.items():
+        if v.dtype == np.uint16:
+            out[k] = _dev_bits(v)
+        else:
+            out[k] = torch.from_numpy(np.ascontiguousarray(v, dtype=np.float32)).cuda()
+    return out
+
+
+def _check(got, want, x0, rows, scale=1.0):
+    g, r, x = got[rows], want[rows], x0[rows]
+    fro = np.linalg.norm(g - r) / np.linalg.norm(r)
+    dfro = np.linalg.norm((g - x) - (r - x)) / np.linalg.norm(r - x)
+    mx = np.abs(g - r).max()
+    assert np.isfinite(g).all()
+    assert fro <= OUT_FRO * scale and dfro <= DELTA_FRO * scale and mx <= MAX_ABS * scale, (fro, dfro, mx)
+
+
+BLOCK_CASES = [
+    ("frame", shp(3, 4, 5, 7, 9)),          # C = 256, T = 68: GEMM row tiles straddle frames, ragged tail
+    ("global", shp(3, 4, 5, 7, 9)),
+    ("register", shp(40, 4, 5, 2, 3)),      # 200 special tokens of 11-token frames
+    ("frame", shp(2, 16, 17, 6, 8)),        # C = 1024, T = 65
+    ("global", shp(2, 16, 17, 6, 8)),
+    ("register", shp(9, 16, 17, 6, 8)),     # 153 special tokens
+    ("global", shp(2, 32, 17, 3, 4)),       # C = 2048 (LayerNorm with 8 chunks per lane)
+]
+
+
+@pytest.mark.parametrize("mode,shape", BLOCK_CASES, ids=[f"{m}-S{s.S}T{s.T}H{s.H}" for m, s in BLOCK_CASES])
+def test_block_matches_oracle(mode, shape):
+    import torch
+    import vit_attention_b200 as V
+    w = W.make_transformer_block_weights(shape.H, 50 + shape.H)
+    x = W.make_tokens(shape, 60 + shape.T)
+    xd = _dev_bits(x).clone()
+    ws = torch.empty(V.vggt_block_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+    V.vggt_block_forward(mode, shape, xd, _dev_weights(w), EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    got = xd.float().cpu().numpy().astype(np.float64)
+    want = O.block_forward(mode, shape, x, w, EPS)
+    x0 = O.bf16_to_f64(x)
+    rows = O.register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T)
+    _check(got, want, x0, rows)
+    if mode == "register":   # patch rows untouched, bit for bit
+        patch = np.setdiff1d(np.arange(shape.S * shape.T), rows)
+        assert np.array_equal(xd.view(torch.int16).cpu().numpy().view(np.uint16)[patch], x[patch])
+
+
+def test_zero_layerscale_leaves_x_bit_identical():
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(2, 4, 5, 7, 9)
+    w = W.make_transformer_block_weights(shape.H, 70)
+    w["ls1"] = np.zeros_like(w["ls1"])
+    w["ls2"] = np.zeros_like(w["ls2"])
+    x = W.make_tokens(shape, 71)
+    xd = _dev_bits(x).clone()
+    ws = torch.empty(V.vggt_block_workspace_size(shape, "global"), dtype=torch.uint8, device="cuda")
+    V.vggt_block_forward("global", shape, xd, _dev_weights(w), EPS, ws)
+    assert np.array_equal(xd.view(torch.int16).cpu().numpy().view(np.uint16), x)
+
+
+def test_aggregator_two_layers_with_a_register_layer():
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(6, 4, 5, 4, 5)     # C = 256, T = 25
+    fw = [W.make_transformer_block_weights(shape.H, 80 + l) for l in range(2)]
+    iw = [W.make_transformer_block_weights(shape.H, 90 + l) for l in range(2)]
+    x = W.make_tokens(shape, 99)
+    xd = _dev_bits(x).clone()
+    ws = torch.empty(V.vggt_aggregator_workspace_size(shape), dtype=torch.uint8, device="cuda")
+    V.vggt_aggregator_forward(shape, xd, [_dev_weights(w) for w in fw], [_dev_weights(w) for w in iw], [1], EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    got = xd.float().cpu().numpy().astype(np.float64)
+    want = O.aggregator_forward(shape, x, fw, iw, [1], EPS)
+    _check(got, want, O.bf16_to_f64(x), np.arange(shape.S * shape.T), scale=2.0)
+
+
+def test_block_argument_errors():
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(2, 4, 5, 7, 9)
+    w = _dev_weights(W.make_transformer_block_weights(shape.H, 70))
+    x = _dev_bits(W.make_tokens(shape, 71))
+    ws = torch.empty(V.vggt_block_workspace_size(shape, "frame"), dtype=torch.uint8, device="cuda")
+    with pytest.raises(V.VggtAttnError) as e:        # C = 128: not a multiple of 256
+        V.vggt_block_forward("frame", shp(2, 2, 5, 7, 9), x, w, EPS, ws)
+    assert e.value.code == V.ERR_UNSUPPORTED_SHAPE
+    with pytest.raises(V.VggtAttnError) as e:
+        V.vggt_block_forward("frame", shape, x, w, EPS, ws, workspace_bytes=ws.numel() - 1)
+    assert e.value.code == V.ERR_WORKSPACE_TOO_SMALL
+    with pytest.raises(V.VggtAttnError) as e:
+        V.vggt_block_forward("frame", shape, x, dict(w, ls1=None), EPS, ws)
+    assert e.value.code == V.ERR_INVALID_ARG
+    with pytest.raises(V.VggtAttnError) as e:        # x inside the workspace
+        V.vggt_block_forward("frame", shape, ws, w, EPS, ws)
+    assert e.value.code == V.ERR_INVALID_ARG

@@ -36,6 +36,15 @@ class vggt_attn_shape(ctypes.Structure):  # noqa: N801 - C name
                 ("ln_eps", ctypes.c_float), ("rope_base", ctypes.c_float), ("softmax_scale", ctypes.c_float)]
 
 
+BLOCK_WEIGHT_FIELDS = ("norm1_gamma", "norm1_beta", "w_qkv", "b_qkv", "q_gamma", "q_beta", "k_gamma", "k_beta",
+                       "w_proj", "b_proj", "ls1", "norm2_gamma", "norm2_beta", "w_fc1", "b_fc1", "w_fc2", "b_fc2",
+                       "ls2")
+
+
+class vggt_block_weights(ctypes.Structure):  # noqa: N801 - C name
+    _fields_ = [(f, ctypes.c_void_p) for f in BLOCK_WEIGHT_FIELDS]
+
+
 class VggtAttnError(RuntimeError):
     def __init__(self, code: int, where: str):
         self.code = code
@@ -67,6 +76,13 @@ _SIGNATURES = {
     "vggt_attn_qkv_proj": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
     "vggt_attn_block": (_int, [_int, _shape_p, _vp, _vp, _fp, _fp, _fp, _fp, _fp, _vp, _fp, _vp, _vp, _vp, _vp, _sz,
                                _vp]),
+    "vggt_block_workspace_size": (_sz, [_shape_p, _int]),
+    "vggt_block_forward": (_int, [_int, _shape_p, _vp, ctypes.POINTER(vggt_block_weights), ctypes.c_float, _vp, _sz,
+                                  _vp]),
+    "vggt_aggregator_workspace_size": (_sz, [_shape_p]),
+    "vggt_aggregator_forward": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
+                                       ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int), _int,
+                                       ctypes.c_float, _vp, _sz, _vp]),
     "vggt_attn_sga_workspace_size": (_sz, [_shape_p, _int, _int]),
     "vggt_attn_global_sga": (_int, [_shape_p, _int, _int, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
 }
@@ -237,3 +253,44 @@ def vggt_attn_global_sga(shape, s_h, s_w, qkv, q_gamma, q_beta, k_gamma, k_beta,
                                    _ptr(k_gamma), _ptr(k_beta), _ptr(out), _ptr(workspace),
                                    _nbytes(workspace, workspace_bytes), _stream(stream))
     _check(rc, "vggt_attn_global_sga")
+
+
+def make_block_weights(w) -> vggt_block_weights:
+    """C struct of device addresses from a mapping with the struct's field names (tensors, ints or None)."""
+    if isinstance(w, vggt_block_weights):
+        return w
+    return vggt_block_weights(*[_ptr(w.get(f)) for f in BLOCK_WEIGHT_FIELDS])
+
+
+def vggt_block_workspace_size(shape, mode) -> int:
+    mode = MODES.get(mode, mode)
+    return _lib.vggt_block_workspace_size(ctypes.byref(make_shape(shape)), mode)
+
+
+def vggt_block_forward(mode, shape, x, weights, norm_eps, workspace, workspace_bytes=None, stream=None):
+    """One pre-norm transformer block applied in place to x [S][T][C] (bf16)."""
+    mode = MODES.get(mode, mode)
+    w = make_block_weights(weights)
+    rc = _lib.vggt_block_forward(mode, ctypes.byref(make_shape(shape)), _ptr(x), ctypes.byref(w), norm_eps,
+                                 _ptr(workspace), _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_block_forward")
+
+
+def vggt_aggregator_workspace_size(shape) -> int:
+    return _lib.vggt_aggregator_workspace_size(ctypes.byref(make_shape(shape)))
+
+
+def vggt_aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, norm_eps, workspace,
+                            workspace_bytes=None, stream=None):
+    """Alternating frame / inter-frame blocks applied in place to x; inter-frame blocks of the layers in
+    register_layers run in register mode, the others in global mode."""
+    n = len(frame_blocks)
+    if len(inter_blocks) != n:
+        raise ValueError("frame_blocks and inter_blocks must have one entry per layer")
+    fb = (vggt_block_weights * max(n, 1))(*[make_block_weights(w) for w in frame_blocks])
+    ib = (vggt_block_weights * max(n, 1))(*[make_block_weights(w) for w in inter_blocks])
+    regs = (ctypes.c_int * max(len(register_layers), 1))(*register_layers)
+    rc = _lib.vggt_aggregator_forward(ctypes.byref(make_shape(shape)), _ptr(x), fb, ib, n, regs,
+                                      len(register_layers), norm_eps, _ptr(workspace),
+                                      _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_aggregator_forward")

@@ -1,6 +1,9 @@
 """Build libvggt_attn.so in-tree for sm_100a (B200).
 
-    python -m vit_attention_b200.build        # or: python vit_attention_b200/build.py
+    python vit_attention_b200/build.py [--force]
+
+(Run as a file, not through the package: the package's __init__ loads the
+library this script builds.)
 
 nvcc cross-compiles without a GPU.  The CUDA runtime is linked statically, so
 the library only needs the NVIDIA driver at run time.
@@ -16,9 +19,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libvggt_attn.so")
 SOURCES = [os.path.join(HERE, "csrc", "vggt_attn.cu")]
-DEPENDS = SOURCES + [os.path.join(HERE, "csrc", f) for f in
-                     ("attention_sm100.cuh", "attention_frame_persistent.cuh", "linear_sm100.cuh", "prologue.cuh", "sga.cuh", "common.cuh", "ptx_sm100.cuh")] + \
-          [os.path.join(ROOT, "include", "vggt_attn.h")]
+DEPENDS = SOURCES + sorted(os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))
+                           if f.endswith(".cuh")) + [os.path.join(ROOT, "include", "vggt_attn.h")]
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

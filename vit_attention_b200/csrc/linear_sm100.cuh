@@ -5,8 +5,12 @@
 // alternating-attention layer projects its 1024 channels to q, k, v and its
 // attention output back to 1024 channels.)
 //
-// Two epilogues:
+// Epilogues (the template argument EPI picks one; each is its own kernel):
 //   plain  -- bf16(Y) into y[M][N] (the output projection, or an unfused qkv);
+//   gelu   -- bf16(GELU(Y)) into y (the MLP's first layer; exact erf form);
+//   resid  -- y = r + ls * Y with r a bf16 [M][N] residual and ls a per-column
+//             LayerScale vector, into y (may be r itself: each element is read
+//             by the thread that then writes it, before the chunk's store);
 //   qkv    -- the QKV projection of a frame or global attention block: the
 //             columns of a 64-wide head slice of q or k go through the QK
 //             LayerNorm, the 2D RoPE and (q) the softmax scale in fp32 straight
@@ -63,6 +67,7 @@ constexpr int THREADS = 256;
 constexpr uint32_t TMEM_COLS = 512;                    // two 256-column accumulators
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
 constexpr int REGS_AT_LAUNCH = 168;
+enum { EPI_STD = 0, EPI_GELU = 1, EPI_RESID = 2 };     // EPI_STD: plain or qkv (LinearParams::fused)
 }  // namespace lin
 
 struct LinearParams {
@@ -78,6 +83,9 @@ struct LinearParams {
   const float* beta[2];
   int H, T, n_special, grid_h, grid_w;
   float eps, q_mult, rope_base;
+  // residual epilogue: y = resid + ls * (X W^T + b), resid bf16 [M][N]
+  const uint16_t* resid;
+  const float* ls;             // [N]
 };
 
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int c0, int c1, int c2) {
@@ -126,6 +134,7 @@ __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
 // thread with one TMA store; `chunk` counts the CTA's chunks (barrier phases).
 // Loads of bias, gamma and beta are issued a few at a time, so that the
 // chunk's 64 values are the only large live state.
+template <int EPI>
 __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t acc, int m0, int n0, int row,
                                                 bool leader, uint8_t* stage, uint32_t bar0, volatile int* abort_flag,
                                                 int& chunk, const CUtensorMap* to0, const CUtensorMap* to1,
@@ -149,7 +158,32 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
         v[e + 3] = __float_as_uint(__uint_as_float(v[e + 3]) + bv.w);
       }
     }
-    const int c = p.fused ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
+    if constexpr (EPI == lin::EPI_GELU) {
+#pragma unroll
+      for (int e = 0; e < 64; ++e) {
+        const float x = __uint_as_float(v[e]);
+        v[e] = __float_as_uint(0.5f * x * (1.0f + erff(x * 0.70710678118654752f)));   // x * Phi(x)
+      }
+    }
+    if constexpr (EPI == lin::EPI_RESID) {
+      // Rows past M have no residual (their values are clipped by the store).
+      const uint4* rrow = reinterpret_cast<const uint4*>(p.resid + static_cast<long long>(m) * p.N + col0);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint4 r = m < p.M ? rrow[k] : make_uint4(0u, 0u, 0u, 0u);
+        const float4 l0 = __ldg(reinterpret_cast<const float4*>(p.ls + col0 + 8 * k));
+        const float4 l1 = __ldg(reinterpret_cast<const float4*>(p.ls + col0 + 8 * k + 4));
+        const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+        const float lv[8] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const float r0 = __uint_as_float(rw[i] << 16), r1 = __uint_as_float(rw[i] & 0xFFFF0000u);
+          v[8 * k + 2 * i] = __float_as_uint(r0 + lv[2 * i] * __uint_as_float(v[8 * k + 2 * i]));
+          v[8 * k + 2 * i + 1] = __float_as_uint(r1 + lv[2 * i + 1] * __uint_as_float(v[8 * k + 2 * i + 1]));
+        }
+      }
+    }
+    const int c = (EPI == lin::EPI_STD && p.fused) ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
     const int h = (col0 / 64) % p.H;
     uint4 o[8];
     if (c == 2) {
@@ -160,7 +194,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
         o[k].z = pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]));
         o[k].w = pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
       }
-    } else {
+    } else if constexpr (EPI == lin::EPI_STD) {
       // QK LayerNorm over the head's 64 values (biased variance, two passes;
       // eight partial sums each, then a short tree).
       float ps[8];
@@ -247,7 +281,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
       ok = wait_bounded(bar(BAR_STAGE_FULL), chunk & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
       if (ok) {
         const uint32_t src = smem_addr(stage);
-        if (!p.fused)
+        if (EPI != lin::EPI_STD || !p.fused)
           tma_store_3d(to0, src, col0, m0, 0);          // y [M][N]
         else if (c == 2)
           tma_store_4d(to0, src, 0, h, 2, m0);          // v slot of qkv [M][3][H][64]
@@ -262,6 +296,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
   return true;
 }
 
+template <int EPI>
 __global__ void __launch_bounds__(lin::THREADS, 1)
     linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const __grid_constant__ CUtensorMap tmap_o0, const __grid_constant__ CUtensorMap tmap_o1,
@@ -404,7 +439,7 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-        ok = linear_epilogue(p, tmem + lane_base + ab * BN, m0, n0, row, leader, smem + OFF_STAGE, bar0, abort_flag,
+        ok = linear_epilogue<EPI>(p, tmem + lane_base + ab * BN, m0, n0, row, leader, smem + OFF_STAGE, bar0, abort_flag,
                              chunk, &tmap_o0, &tmap_o1, &tmap_o2, rope_tab);
         tc_fence_before();
         mbar_arrive(bar(BAR_ACC_EMPTY + ab));

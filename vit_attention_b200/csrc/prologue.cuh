@@ -63,7 +63,8 @@ struct PrologueParams {
   const float* beta[2];
   uint16_t* ws_qk[2];     // q, k destinations
   uint16_t* ws_v;         // register mode only
-  int* status;
+  int* status;         // cleared by block 0 when zero_status (the first kernel of a call)
+  int zero_status;
   int n_tok;              // tokens in the mode's token list (< 2^31, checked on the host)
   int T, H, n_special, grid_h, grid_w;
   int mode;               // VGGT_ATTN_FRAME / GLOBAL / REGISTER
@@ -116,7 +117,7 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
     sincos(pos * omega, &s, &c);
     rope_tab[e] = make_float2(static_cast<float>(c), static_cast<float>(s));
   }
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
+  if (p.zero_status && blockIdx.x == 0 && threadIdx.x == 0) {
     p.status[0] = 0;
     p.status[1] = 0;
   }

@@ -12,6 +12,7 @@
 
 #include "attention_frame_persistent.cuh"
 #include "attention_sm100.cuh"
+#include "layernorm.cuh"
 #include "linear_sm100.cuh"
 #include "prologue.cuh"
 #include "sga.cuh"
@@ -131,8 +132,12 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* di
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// clear_status: the prologue is the call's first kernel (the attention entry
+// points); inside a block an earlier kernel has cleared the status word and
+// may already have recorded an error in it.
 int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const float* gq, const float* bq,
-                    const float* gk, const float* bk, const WorkspaceView& w, cudaStream_t stream) {
+                    const float* gk, const float* bk, const WorkspaceView& w, cudaStream_t stream,
+                    bool clear_status = true) {
   const ModeGeometry g = geometry(s, mode);
   vggt::PrologueParams p;
   p.qkv = static_cast<const uint16_t*>(qkv);
@@ -144,6 +149,7 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.ws_qk[1] = w.k;
   p.ws_v = w.v;
   p.status = w.status;
+  p.zero_status = clear_status ? 1 : 0;
   p.n_tok = static_cast<int>(g.n_tok);
   p.T = s->T;
   p.H = s->H;
@@ -487,15 +493,22 @@ int check_linear_dims(long long M, long long N, long long K) {
 
 // Output maps: o0 = y [M][N] (plain) or the v slot of qkv [M][3][H][64]
 // (fused, as (64, H, 3, M)); o1, o2 = the q and k planes [H][M][64] (fused).
+template <int EPI>
+int launch_linear_epi(const vggt::LinearParams& p, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& o0,
+                      const CUtensorMap& o1, const CUtensorMap& o2, int smem, unsigned grid, cudaStream_t stream) {
+  if (cudaFuncSetAttribute(vggt::linear_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  vggt::linear_kernel<EPI><<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, o0, o1, o2, p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
 int launch_linear(vggt::LinearParams p, const void* x, const void* w, const CUtensorMap& o0, const CUtensorMap& o1,
-                  const CUtensorMap& o2, int grid_h, int grid_w, cudaStream_t stream) {
+                  const CUtensorMap& o2, int grid_h, int grid_w, cudaStream_t stream, int epi = vggt::lin::EPI_STD) {
   CUtensorMap mx, mw;
   if (!make_rows_map(&mx, x, p.K, p.M, vggt::lin::BM) || !make_rows_map(&mw, w, p.K, p.N, vggt::lin::BN))
     return VGGT_ATTN_ERR_CUDA;
   const int smem = vggt::linear_smem_bytes(grid_h, grid_w);
   if (smem > 227 * 1024) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
-  if (cudaFuncSetAttribute(vggt::linear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-    return VGGT_ATTN_ERR_CUDA;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
@@ -503,8 +516,11 @@ int launch_linear(vggt::LinearParams p, const void* x, const void* w, const CUte
   const long long tiles = ((p.M + vggt::lin::BM - 1) / vggt::lin::BM) * static_cast<long long>(p.N / vggt::lin::BN);
   const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);   // persistent: one CTA per SM
   p.timeout_ns = kDefaultTimeoutNs;
-  vggt::linear_kernel<<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, o0, o1, o2, p);
-  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+  switch (epi) {
+    case vggt::lin::EPI_GELU: return launch_linear_epi<vggt::lin::EPI_GELU>(p, mx, mw, o0, o1, o2, smem, grid, stream);
+    case vggt::lin::EPI_RESID: return launch_linear_epi<vggt::lin::EPI_RESID>(p, mx, mw, o0, o1, o2, smem, grid, stream);
+    default: return launch_linear_epi<vggt::lin::EPI_STD>(p, mx, mw, o0, o1, o2, smem, grid, stream);
+  }
 }
 
 int check_qkv_proj_args(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
@@ -634,18 +650,23 @@ int launch_special_rows(const void* src, void* dst, int n_rows, long long row_by
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
+// y = epi(x w^T + b) into y [M][N]; EPI_RESID reads resid [M][N] and ls [N].
 int launch_linear_plain(const void* x, const void* w, const float* b, void* y, long long M, long long N, long long K,
-                        int* status, cudaStream_t st) {
+                        int* status, cudaStream_t st, bool zero_status = false, int epi = vggt::lin::EPI_STD,
+                        const void* resid = nullptr, const float* ls = nullptr) {
   vggt::LinearParams p{};
   p.M = static_cast<int>(M);
   p.N = static_cast<int>(N);
   p.K = static_cast<int>(K);
   p.bias = b;
   p.status = status;
+  p.zero_status = zero_status ? 1 : 0;
   p.grid_w = 1;
+  p.resid = static_cast<const uint16_t*>(resid);
+  p.ls = ls;
   CUtensorMap my;
   if (!make_rows_map(&my, y, N, M, vggt::lin::BM)) return VGGT_ATTN_ERR_CUDA;
-  return launch_linear(p, x, w, my, my, my, 0, 0, st);
+  return launch_linear(p, x, w, my, my, my, 0, 0, st, epi);
 }
 
 int check_block_args(int mode, const vggt_attn_shape* s, const void* x, const void* w_qkv, const float* b_qkv,
@@ -698,8 +719,9 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
     uint8_t* ys = as + Ms * row;
     const WorkspaceView wv = workspace_view(&s2, VGGT_ATTN_GLOBAL, workspace);
     if ((rc = launch_special_rows(x, xs, static_cast<int>(Ms), row, shape->n_special, shape->T, true, st))) return rc;
-    if ((rc = launch_linear_plain(xs, w_qkv, b_qkv, qkv, Ms, 3 * C, C, wv.status, st))) return rc;
-    if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, &s2, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st))) return rc;
+    if ((rc = launch_linear_plain(xs, w_qkv, b_qkv, qkv, Ms, 3 * C, C, wv.status, st, true))) return rc;
+    if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, &s2, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st, false)))
+      return rc;
     if ((rc = launch_core(VGGT_ATTN_GLOBAL, &s2, qkv, as, wv, st))) return rc;
     if ((rc = launch_linear_plain(as, w_out, b_out, ys, Ms, C, C, wv.status, st))) return rc;
     return launch_special_rows(ys, y, static_cast<int>(Ms), row, shape->n_special, shape->T, false, st);
@@ -708,8 +730,8 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
   // QKV projection as a plain GEMM into qkv, then the prologue: measured
   // faster than the fused projection (whose LayerNorm/RoPE epilogue, not its
   // products, sets its time) on both the frame and the global workloads.
-  if ((rc = launch_linear_plain(x, w_qkv, b_qkv, qkv, M, 3 * C, C, wv.status, st))) return rc;
-  if ((rc = launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st))) return rc;
+  if ((rc = launch_linear_plain(x, w_qkv, b_qkv, qkv, M, 3 * C, C, wv.status, st, true))) return rc;
+  if ((rc = launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st, false))) return rc;
   if ((rc = launch_core(mode, shape, qkv, attn, wv, st))) return rc;
   return launch_linear_plain(attn, w_out, b_out, y, M, C, C, wv.status, st);
 }
@@ -837,4 +859,229 @@ extern "C" int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s
            g.T, g.n_special, g.grid_w, g.s_h, g.s_w};
   ModeGeometry mg{1, g.N, g.N, 2};
   return launch_core_cfg<vggt::CoreCfg<2, true>>(mg, g.H, mq, mk, mv, p, st);
+}
+
+// ---------------------------------------------------------------------------
+// Transformer blocks and the alternating-attention schedule (VGGT-Omega
+// Aggregator explainer, section 3).
+namespace {
+
+constexpr int kMaxBlockChannels = 2048;   // LayerNorm kernel: up to 8 16-byte chunks per lane
+
+struct BlockLayout {
+  vggt_attn_shape s;        // the shape the block's kernels see (register mode: special tokens only)
+  int mode;                 // the attention mode they run (register mode: global)
+  long long M;              // rows the block processes
+  WorkspaceView att;        // attention workspace (status word first)
+  uint8_t* xs;              // register mode: the gathered rows of x [M][C]
+  uint8_t* h;               // norm output [M][C]
+  uint8_t* big;             // qkv [M][3C] then attention output [M][C]; later the hidden [M][4C]
+  size_t bytes;
+};
+
+BlockLayout block_layout(const vggt_attn_shape* shape, int mode, void* ws) {
+  BlockLayout L{};
+  L.s = *shape;
+  L.mode = mode;
+  if (mode == VGGT_ATTN_REGISTER) {
+    L.s.T = shape->n_special;
+    L.s.grid_h = 0;
+    L.s.grid_w = 0;
+    L.mode = VGGT_ATTN_GLOBAL;
+  }
+  L.M = static_cast<long long>(L.s.S) * L.s.T;
+  const size_t row = static_cast<size_t>(shape->H) * 64 * 2;
+  L.att = workspace_view(&L.s, L.mode, ws);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = L.att.bytes;
+  if (mode == VGGT_ATTN_REGISTER) {
+    L.xs = base + off;
+    off += align256(L.M * row);
+  }
+  L.h = base + off;
+  off += align256(L.M * row);
+  L.big = base + off;
+  off += align256(L.M * 4 * row);
+  L.bytes = off;
+  return L;
+}
+
+int check_block_shape(const vggt_attn_shape* s, int mode) {
+  int rc = check_shape(s, mode);
+  if (rc) return rc;
+  const long long C = static_cast<long long>(s->H) * 64;
+  if (C % 256 || C > kMaxBlockChannels) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  const long long M = static_cast<long long>(s->S) * (mode == VGGT_ATTN_REGISTER ? s->n_special : s->T);
+  if ((rc = check_linear_dims(M, 4 * C, C)) || (rc = check_linear_dims(M, C, 4 * C))) return rc;
+  return VGGT_ATTN_OK;
+}
+
+bool vec_ok(const float* p, bool optional) { return p ? aligned(p, 16) : optional; }
+
+int check_block_weights(const vggt_block_weights* w, long long C, const void* x, size_t x_bytes, const void* ws,
+                        size_t ws_bytes) {
+  if (!w) return VGGT_ATTN_ERR_INVALID_ARG;
+  const float* req[] = {w->norm1_gamma, w->norm1_beta, w->q_gamma, w->q_beta, w->k_gamma,
+                        w->k_beta,      w->ls1,        w->norm2_gamma, w->norm2_beta, w->ls2};
+  for (const float* v : req)
+    if (!v) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!w->w_qkv || !w->w_proj || !w->w_fc1 || !w->w_fc2) return VGGT_ATTN_ERR_INVALID_ARG;
+  for (const float* v : req)
+    if (!vec_ok(v, false)) return VGGT_ATTN_ERR_MISALIGNED;
+  if (!vec_ok(w->b_qkv, true) || !vec_ok(w->b_proj, true) || !vec_ok(w->b_fc1, true) || !vec_ok(w->b_fc2, true))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  if (!aligned(w->w_qkv, 16) || !aligned(w->w_proj, 16) || !aligned(w->w_fc1, 16) || !aligned(w->w_fc2, 16))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t cc = static_cast<size_t>(C) * C * 2;
+  const void* mats[4] = {w->w_qkv, w->w_proj, w->w_fc1, w->w_fc2};
+  const size_t mat_bytes[4] = {3 * cc, cc, 4 * cc, 4 * cc};
+  for (int i = 0; i < 4; ++i)
+    if (overlaps(x, x_bytes, mats[i], mat_bytes[i]) || overlaps(ws, ws_bytes, mats[i], mat_bytes[i]))
+      return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+int launch_layernorm(const void* x, void* y, const float* gamma, const float* beta, long long M, long long C,
+                     float eps, int* status, bool zero_status, cudaStream_t st) {
+  vggt::LayerNormParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.y = static_cast<uint16_t*>(y);
+  p.gamma = gamma;
+  p.beta = beta;
+  p.M = M;
+  p.eps = eps;
+  p.status = status;
+  p.zero_status = zero_status ? 1 : 0;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+    return VGGT_ATTN_ERR_CUDA;
+  long long blocks = (M + 7) / 8;                    // 8 rows (warps) per block
+  const long long cap = static_cast<long long>(sms) * 8;
+  if (blocks > cap) blocks = cap;
+  const unsigned grid = static_cast<unsigned>(blocks);
+  switch (C / 256) {
+    case 1: vggt::layernorm_rows_kernel<1><<<grid, 256, 0, st>>>(p); break;
+    case 2: vggt::layernorm_rows_kernel<2><<<grid, 256, 0, st>>>(p); break;
+    case 3: vggt::layernorm_rows_kernel<3><<<grid, 256, 0, st>>>(p); break;
+    case 4: vggt::layernorm_rows_kernel<4><<<grid, 256, 0, st>>>(p); break;
+    case 5: vggt::layernorm_rows_kernel<5><<<grid, 256, 0, st>>>(p); break;
+    case 6: vggt::layernorm_rows_kernel<6><<<grid, 256, 0, st>>>(p); break;
+    case 7: vggt::layernorm_rows_kernel<7><<<grid, 256, 0, st>>>(p); break;
+    case 8: vggt::layernorm_rows_kernel<8><<<grid, 256, 0, st>>>(p); break;
+    default: return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  }
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
+}
+
+// The kernels of one block; arguments already validated.
+// clear_status: this block's first kernel clears the status word (the first
+// block of a call); later blocks keep what earlier ones recorded.
+int run_block(int mode, const vggt_attn_shape* shape, void* x, const vggt_block_weights* w, float eps, void* ws,
+              bool clear_status, cudaStream_t st) {
+  const BlockLayout L = block_layout(shape, mode, ws);
+  const long long C = static_cast<long long>(shape->H) * 64, M = L.M;
+  int* status = L.att.status;
+  int rc;
+  void* xb = x;
+  if (mode == VGGT_ATTN_REGISTER) {
+    if ((rc = launch_special_rows(x, L.xs, static_cast<int>(M), C * 2, shape->n_special, shape->T, true, st)))
+      return rc;
+    xb = L.xs;
+  }
+  uint8_t* qkv = L.big;
+  uint8_t* att = L.big + static_cast<size_t>(M) * 3 * C * 2;
+  if ((rc = launch_layernorm(xb, L.h, w->norm1_gamma, w->norm1_beta, M, C, eps, status, clear_status, st)))
+    return rc;
+  if ((rc = launch_linear_plain(L.h, w->w_qkv, w->b_qkv, qkv, M, 3 * C, C, status, st))) return rc;
+  if ((rc = launch_prologue(L.mode, &L.s, qkv, w->q_gamma, w->q_beta, w->k_gamma, w->k_beta, L.att, st, false)))
+    return rc;
+  if ((rc = launch_core(L.mode, &L.s, qkv, att, L.att, st))) return rc;
+  if ((rc = launch_linear_plain(att, w->w_proj, w->b_proj, xb, M, C, C, status, st, false, vggt::lin::EPI_RESID, xb,
+                                w->ls1)))
+    return rc;
+  if ((rc = launch_layernorm(xb, L.h, w->norm2_gamma, w->norm2_beta, M, C, eps, status, false, st))) return rc;
+  if ((rc = launch_linear_plain(L.h, w->w_fc1, w->b_fc1, L.big, M, 4 * C, C, status, st, false, vggt::lin::EPI_GELU)))
+    return rc;
+  if ((rc = launch_linear_plain(L.big, w->w_fc2, w->b_fc2, xb, M, C, 4 * C, status, st, false, vggt::lin::EPI_RESID,
+                                xb, w->ls2)))
+    return rc;
+  if (mode == VGGT_ATTN_REGISTER)
+    return launch_special_rows(L.xs, x, static_cast<int>(M), C * 2, shape->n_special, shape->T, false, st);
+  return VGGT_ATTN_OK;
+}
+
+int check_block_common(const vggt_attn_shape* shape, void* x, void* ws, size_t ws_bytes, size_t need) {
+  if (!x || !ws) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(ws, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  if (ws_bytes < need) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  const size_t x_bytes = static_cast<size_t>(shape->S) * shape->T * shape->H * 64 * 2;
+  if (overlaps(x, x_bytes, ws, ws_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  return VGGT_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" size_t vggt_block_workspace_size(const vggt_attn_shape* shape, int mode) {
+  if (check_block_shape(shape, mode) != VGGT_ATTN_OK) return 0;
+  return block_layout(shape, mode, nullptr).bytes;
+}
+
+extern "C" int vggt_block_forward(int mode, const vggt_attn_shape* shape, void* x, const vggt_block_weights* w,
+                                  float norm_eps, void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_block_shape(shape, mode);
+  if (rc) return rc;
+  if (!std::isfinite(norm_eps) || !(norm_eps > 0.f)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_block_common(shape, x, workspace, workspace_bytes, vggt_block_workspace_size(shape, mode))))
+    return rc;
+  const size_t x_bytes = static_cast<size_t>(shape->S) * shape->T * shape->H * 64 * 2;
+  if ((rc = check_block_weights(w, static_cast<long long>(shape->H) * 64, x, x_bytes, workspace, workspace_bytes)))
+    return rc;
+  if ((rc = check_device())) return rc;
+  return run_block(mode, shape, x, w, norm_eps, workspace, true, static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" size_t vggt_aggregator_workspace_size(const vggt_attn_shape* shape) {
+  size_t need = 0;
+  for (int mode : {VGGT_ATTN_FRAME, VGGT_ATTN_GLOBAL, VGGT_ATTN_REGISTER}) {
+    if (mode == VGGT_ATTN_REGISTER && (!shape || shape->n_special < 1)) continue;
+    const size_t b = vggt_block_workspace_size(shape, mode);
+    if (b == 0) return 0;
+    need = std::max(need, b);
+  }
+  return need;
+}
+
+extern "C" int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_block_weights* frame_blocks,
+                                       const vggt_block_weights* inter_blocks, int n_layers,
+                                       const int* register_layers, int n_register, float norm_eps, void* workspace,
+                                       size_t workspace_bytes, void* cuda_stream) {
+  if (n_layers < 0 || n_register < 0 || (n_register > 0 && !register_layers)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (n_layers > 0 && (!frame_blocks || !inter_blocks)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(norm_eps) || !(norm_eps > 0.f)) return VGGT_ATTN_ERR_INVALID_ARG;
+  int rc;
+  if ((rc = check_block_shape(shape, VGGT_ATTN_FRAME)) || (rc = check_block_shape(shape, VGGT_ATTN_GLOBAL)))
+    return rc;
+  for (int i = 0; i < n_register; ++i)
+    if (register_layers[i] < 0 || register_layers[i] >= n_layers) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (n_register > 0 && (rc = check_block_shape(shape, VGGT_ATTN_REGISTER))) return rc;
+  if ((rc = check_block_common(shape, x, workspace, workspace_bytes, vggt_aggregator_workspace_size(shape))))
+    return rc;
+  const long long C = static_cast<long long>(shape->H) * 64;
+  const size_t x_bytes = static_cast<size_t>(shape->S) * shape->T * C * 2;
+  for (int l = 0; l < n_layers; ++l)
+    if ((rc = check_block_weights(&frame_blocks[l], C, x, x_bytes, workspace, workspace_bytes)) ||
+        (rc = check_block_weights(&inter_blocks[l], C, x, x_bytes, workspace, workspace_bytes)))
+      return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  for (int l = 0; l < n_layers; ++l) {
+    bool reg = false;
+    for (int i = 0; i < n_register; ++i) reg = reg || register_layers[i] == l;
+    if ((rc = run_block(VGGT_ATTN_FRAME, shape, x, &frame_blocks[l], norm_eps, workspace, l == 0, st))) return rc;
+    if ((rc = run_block(reg ? VGGT_ATTN_REGISTER : VGGT_ATTN_GLOBAL, shape, x, &inter_blocks[l], norm_eps, workspace,
+                        false, st)))
+      return rc;
+  }
+  return VGGT_ATTN_OK;
 }
