@@ -22,6 +22,7 @@ the fp64 oracle instead (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -382,6 +383,7 @@ def run_ours(args):
     blocks = {}
     if not args.no_blocks:
         blocks = block_timings(V, device, stream)
+        blocks["transformer"] = transformer_timings(V, device, stream)
     sga = {}
     if not args.no_modes:
         sga = sga_timings(V, device, stream, qkv, prm, out, ms / args.steps)
@@ -506,6 +508,79 @@ def block_timings(V, device, stream):
         entry["qkv_proj_fused_tflops"] = 2.0 * M * 3 * C * C / (entry["qkv_proj_fused_ms"] / 1000) / 1e12
         del x, qkv, attn, y, ws
     res["layer_S500_register_plus_frame_block_ms"] = res["register_S500"]["block_ms"] + res["frame_S500"]["block_ms"]
+    return res
+
+
+def random_block_weights(H: int, g, device):
+    """Device-drawn weights of one transformer block (the oracle's recipe: N(0, 1/fan_in) bf16 matrices,
+    gammas and LayerScales 1 + 0.1 N(0, 1), betas and biases 0.1 N(0, 1))."""
+    import torch
+    C = H * 64
+
+    def mat(n_out, n_in):
+        return (torch.randn((n_out, n_in), generator=g, device=device) / n_in ** 0.5).to(torch.bfloat16)
+
+    def vec(n, centre):
+        return centre + 0.1 * torch.randn(n, generator=g, device=device)
+
+    return dict(norm1_gamma=vec(C, 1.0), norm1_beta=vec(C, 0.0), w_qkv=mat(3 * C, C), b_qkv=vec(3 * C, 0.0),
+                q_gamma=vec(C, 1.0), q_beta=vec(C, 0.0), k_gamma=vec(C, 1.0), k_beta=vec(C, 0.0),
+                w_proj=mat(C, C), b_proj=vec(C, 0.0), ls1=vec(C, 1.0), norm2_gamma=vec(C, 1.0),
+                norm2_beta=vec(C, 0.0), w_fc1=mat(4 * C, C), b_fc1=vec(4 * C, 0.0), w_fc2=mat(C, 4 * C),
+                b_fc2=vec(C, 0.0), ls2=vec(C, 1.0))
+
+
+def transformer_timings(V, device, stream):
+    """Whole transformer blocks (LayerNorm, QKV GEMM, attention, projection + LayerScale residual,
+    LayerNorm, fc1 + GELU, fc2 + LayerScale residual; vggt_block_forward) per mode at S=100 and S=500,
+    the two kinds of layer (frame + global, frame + register), and the 24-layer alternating schedule
+    (register blocks at layers 2, 6, 9, 14, 20; vggt_aggregator_forward) at S=100 (device-drawn inputs,
+    random weights of the model's shapes)."""
+    import torch
+    res = {}
+    g = torch.Generator(device=device)
+    g.manual_seed(8765)
+    eps = 1e-6
+    for idx in (3, 4):
+        shape = W.workload(idx).shape
+        M, C = shape.S * shape.T, shape.H * 64
+        x = torch.randn((M, C), generator=g, device=device).to(torch.bfloat16)
+        ws = torch.empty(V.vggt_aggregator_workspace_size(shape), dtype=torch.uint8, device=device)
+        w = random_block_weights(shape.H, g, device)
+        entry = {}
+        for mode in ("frame", "global", "register"):
+            if idx == 4 and mode == "global":
+                continue                        # S=500 runs register layers only
+            fn = lambda m=mode: V.vggt_block_forward(m, shape, x, w, eps, ws, None, stream)  # noqa: E731
+            fn()
+            entry[f"{mode}_block_ms"] = cuda_time_ms(fn, stream, 3 if mode == "global" else 5)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        if idx == 3:
+            entry["global_layer_ms"] = entry["frame_block_ms"] + entry["global_block_ms"]
+            n = 24
+            fws = [random_block_weights(shape.H, g, device) for _ in range(n)]
+            iws = [random_block_weights(shape.H, g, device) for _ in range(n)]
+            regs = [2, 6, 9, 14, 20]
+            agg = lambda: V.vggt_aggregator_forward(shape, x, fws, iws, regs, eps, ws, None, stream)  # noqa: E731
+            agg()
+            entry["aggregator_24_layers_ms"] = cuda_time_ms(agg, stream, 1)
+            assert V.vggt_attn_read_status(ws, stream) == 0
+            del fws, iws
+        entry["register_layer_ms"] = entry["frame_block_ms"] + entry["register_block_ms"]
+        del x, ws, w
+        # Camera-head trunk: 4 blocks over the S x 17 special tokens of the last layer's
+        # 2 x 1024-wide features (32 heads of 64).
+        fshape = dataclasses.replace(shape, H=2 * shape.H)
+        feats = torch.randn((M, 2 * C), generator=g, device=device).to(torch.bfloat16)
+        tok = torch.empty((shape.S * shape.n_special, 2 * C), dtype=torch.bfloat16, device=device)
+        ws = torch.empty(V.vggt_camera_trunk_workspace_size(fshape), dtype=torch.uint8, device=device)
+        cws = [random_block_weights(fshape.H, g, device) for _ in range(4)]
+        cam = lambda: V.vggt_camera_trunk_forward(fshape, feats, tok, cws, eps, ws, None, stream)  # noqa: E731
+        cam()
+        entry["camera_trunk_4_blocks_ms"] = cuda_time_ms(cam, stream, 5)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        res[f"S{shape.S}"] = entry
+        del feats, tok, ws, cws
     return res
 
 

@@ -333,6 +333,28 @@ int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_bl
                             int n_register, float norm_eps, void* workspace, size_t workspace_bytes,
                             void* cuda_stream);
 
+/* ------------------------------------------------------------------------
+ * Camera-head trunk (VGGT-Omega Aggregator explainer, section 4: the camera
+ * head takes the first 17 tokens of every frame -- camera and register
+ * tokens -- from the last layer's features and mixes them across frames once
+ * more with 4 self-attention blocks before reading out each frame's camera).
+ *
+ * vggt_camera_trunk_forward: gathers rows t < n_special of every frame of
+ * feats (bf16 [S][T][Cf], Cf = 64 Hf, a multiple of 256, at most 2048; the
+ * last layer's concatenated frame and global features, Cf = 2048 for the
+ * 1024-channel backbone) into tokens (bf16 [S n_special][Cf], caller-owned),
+ * then applies n_blocks transformer blocks (vggt_block_forward, global mode
+ * over the S n_special tokens, which carry no RoPE position) to tokens in
+ * place.  shape describes feats: shape->H = Hf, and its S, T, n_special, grid
+ * and epsilons are those of the backbone.  blocks is a host array of n_blocks
+ * weight sets of width Cf.  Workspace: vggt_camera_trunk_workspace_size(shape)
+ * bytes.  Asynchronous on cuda_stream, validates every argument before
+ * enqueueing anything, allocates nothing. */
+size_t vggt_camera_trunk_workspace_size(const vggt_attn_shape* shape);
+int vggt_camera_trunk_forward(const vggt_attn_shape* shape, const void* feats, void* tokens,
+                              const vggt_block_weights* blocks, int n_blocks, float norm_eps,
+                              void* workspace, size_t workspace_bytes, void* cuda_stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -52,7 +52,9 @@ from .attention import (  # noqa: F401
 from .projection import attention_block, linear, projected_qkv  # noqa: F401
 from .sga import attn_global_sga, sga_kept_tokens  # noqa: F401
 from .block import (  # noqa: F401
+    CAMERA_TRUNK_BLOCKS,
     N_LAYERS,
+    camera_trunk_forward,
     REGISTER_LAYERS,
     aggregator_forward,
     block_forward,

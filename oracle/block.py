@@ -11,6 +11,9 @@ Source, cited by page title and section:
        Q/K normalisation together with LayerScale (initial value 1e-5).
   [P1] section 2: the patch tokens come from a DINO-style ViT, whose block
        the Aggregator's blocks follow.
+  [P1] section 4: the camera head takes the first 17 tokens (camera +
+       registers) of every frame from the last layer and mixes them across
+       frames again with 4 self-attention blocks.
 
 Readings where the page is silent (listed in the design doc):
   * A block is the pre-norm transformer block of a DINO-style ViT:
@@ -23,6 +26,11 @@ Readings where the page is silent (listed in the design doc):
     acts on the special tokens only; patch tokens pass through unchanged.
   * The attention inside a block is the core's (QK-LayerNorm, RoPE on patch
     tokens, softmax attention in the block's mode) on the block's own qkv.
+  * The camera head's blocks are blocks of the same form over the S x 17
+    special tokens of the last layer's features (all frames attend to each
+    other; special tokens carry no RoPE position), of the features' width
+    (2 x 1024 for the concatenated frame and global outputs) with 64-wide
+    heads.
 """
 from __future__ import annotations
 
@@ -85,4 +93,18 @@ def aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, no
     for l, (fw, iw) in enumerate(zip(frame_blocks, inter_blocks)):
         y = block_forward("frame", shape, y, fw, norm_eps)
         y = block_forward("register" if l in register_layers else "global", shape, y, iw, norm_eps)
+    return y
+
+
+CAMERA_TRUNK_BLOCKS = 4                  # [P1] section 4
+
+
+def camera_trunk_forward(shape, feats, blocks, norm_eps: float) -> np.ndarray:
+    """The special tokens of every frame of feats ``[S*T, C]``, then each block in
+    turn with attention among all of them.  Returns fp64 ``[S*n_special, C]``."""
+    x = bf16_to_f64(feats) if feats.dtype == np.uint16 else np.asarray(feats, np.float64)
+    y = x[register_tokens(shape)]
+    tok_shape = type(shape)(**{**shape.__dict__, "T": shape.n_special, "grid_h": 0, "grid_w": 0})
+    for w in blocks:
+        y = block_forward("global", tok_shape, y, w, norm_eps)
     return y

@@ -132,3 +132,20 @@ def test_block_argument_errors():
     with pytest.raises(V.VggtAttnError) as e:        # x inside the workspace
         V.vggt_block_forward("frame", shape, ws, w, EPS, ws)
     assert e.value.code == V.ERR_INVALID_ARG
+
+
+def test_camera_trunk_four_blocks():
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(10, 32, 17, 2, 3)     # features of width 2048, 17 special tokens in 23-token frames
+    blocks = [W.make_transformer_block_weights(shape.H, 110 + b) for b in range(4)]
+    feats = W.make_tokens(shape, 120)
+    fd = _dev_bits(feats)
+    tok = torch.empty((shape.S * shape.n_special, shape.H * 64), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(V.vggt_camera_trunk_workspace_size(shape), dtype=torch.uint8, device="cuda")
+    V.vggt_camera_trunk_forward(shape, fd, tok, [_dev_weights(w) for w in blocks], EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    got = tok.float().cpu().numpy().astype(np.float64)
+    want = O.camera_trunk_forward(shape, feats, blocks, EPS)
+    x0 = O.bf16_to_f64(feats)[O.register_tokens(shape)]
+    _check(got, want, x0, np.arange(len(want)), scale=2.0)

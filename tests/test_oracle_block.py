@@ -124,3 +124,13 @@ def test_aggregator_schedule(wts, x):
     y = O.block_forward("register", SHAPE, y, wts, EPS)
     np.testing.assert_array_equal(got, y)
     assert O.REGISTER_LAYERS == (2, 6, 9, 14, 20) and O.N_LAYERS == 24
+
+
+def test_camera_trunk_reduces_to_register_blocks(wts, x):
+    sp = O.register_tokens(SHAPE)
+    np.testing.assert_array_equal(O.camera_trunk_forward(SHAPE, x, [], EPS), O.bf16_to_f64(x)[sp])
+    w2 = W.make_transformer_block_weights(SHAPE.H, 45)
+    y = O.block_forward("register", SHAPE, x, wts, EPS)
+    y = O.block_forward("register", SHAPE, y, w2, EPS)
+    np.testing.assert_allclose(O.camera_trunk_forward(SHAPE, x, [wts, w2], EPS), y[sp], rtol=1e-12, atol=1e-12)
+    assert O.CAMERA_TRUNK_BLOCKS == 4

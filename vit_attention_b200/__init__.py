@@ -83,6 +83,9 @@ _SIGNATURES = {
     "vggt_aggregator_forward": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
                                        ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int), _int,
                                        ctypes.c_float, _vp, _sz, _vp]),
+    "vggt_camera_trunk_workspace_size": (_sz, [_shape_p]),
+    "vggt_camera_trunk_forward": (_int, [_shape_p, _vp, _vp, ctypes.POINTER(vggt_block_weights), _int,
+                                         ctypes.c_float, _vp, _sz, _vp]),
     "vggt_attn_sga_workspace_size": (_sz, [_shape_p, _int, _int]),
     "vggt_attn_global_sga": (_int, [_shape_p, _int, _int, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
 }
@@ -294,3 +297,18 @@ def vggt_aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layer
                                       len(register_layers), norm_eps, _ptr(workspace),
                                       _nbytes(workspace, workspace_bytes), _stream(stream))
     _check(rc, "vggt_aggregator_forward")
+
+
+def vggt_camera_trunk_workspace_size(shape) -> int:
+    return _lib.vggt_camera_trunk_workspace_size(ctypes.byref(make_shape(shape)))
+
+
+def vggt_camera_trunk_forward(shape, feats, tokens, blocks, norm_eps, workspace, workspace_bytes=None, stream=None):
+    """Gather the special tokens of feats [S][T][C] into tokens [S*n_special][C], then apply the blocks
+    (global attention among those tokens) to tokens in place."""
+    n = len(blocks)
+    arr = (vggt_block_weights * max(n, 1))(*[make_block_weights(w) for w in blocks])
+    rc = _lib.vggt_camera_trunk_forward(ctypes.byref(make_shape(shape)), _ptr(feats), _ptr(tokens), arr, n,
+                                        norm_eps, _ptr(workspace), _nbytes(workspace, workspace_bytes),
+                                        _stream(stream))
+    _check(rc, "vggt_camera_trunk_forward")

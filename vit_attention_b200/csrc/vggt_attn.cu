@@ -1085,3 +1085,52 @@ extern "C" int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, co
   }
   return VGGT_ATTN_OK;
 }
+
+// ---------------------------------------------------------------------------
+// Camera-head trunk (VGGT-Omega Aggregator explainer, section 4).
+namespace {
+
+vggt_attn_shape camera_trunk_shape(const vggt_attn_shape* s) {
+  vggt_attn_shape c = *s;
+  c.T = s->n_special;
+  c.grid_h = 0;
+  c.grid_w = 0;
+  return c;
+}
+
+}  // namespace
+
+extern "C" size_t vggt_camera_trunk_workspace_size(const vggt_attn_shape* shape) {
+  if (!shape || shape->n_special < 1 || check_shape(shape, VGGT_ATTN_REGISTER) != VGGT_ATTN_OK) return 0;
+  const vggt_attn_shape c = camera_trunk_shape(shape);
+  return vggt_block_workspace_size(&c, VGGT_ATTN_GLOBAL);
+}
+
+extern "C" int vggt_camera_trunk_forward(const vggt_attn_shape* shape, const void* feats, void* tokens,
+                                         const vggt_block_weights* blocks, int n_blocks, float norm_eps,
+                                         void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_shape(shape, VGGT_ATTN_REGISTER);
+  if (rc) return rc;
+  if (n_blocks < 0 || (n_blocks > 0 && !blocks) || !feats) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!std::isfinite(norm_eps) || !(norm_eps > 0.f)) return VGGT_ATTN_ERR_INVALID_ARG;
+  const vggt_attn_shape c = camera_trunk_shape(shape);
+  if ((rc = check_block_shape(&c, VGGT_ATTN_GLOBAL))) return rc;
+  if (!aligned(feats, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  if ((rc = check_block_common(&c, tokens, workspace, workspace_bytes, vggt_camera_trunk_workspace_size(shape))))
+    return rc;
+  const long long C = static_cast<long long>(shape->H) * 64;
+  const size_t feats_bytes = static_cast<size_t>(shape->S) * shape->T * C * 2;
+  const size_t tok_bytes = static_cast<size_t>(c.S) * c.T * C * 2;
+  if (overlaps(feats, feats_bytes, tokens, tok_bytes) || overlaps(feats, feats_bytes, workspace, workspace_bytes))
+    return VGGT_ATTN_ERR_INVALID_ARG;
+  for (int b = 0; b < n_blocks; ++b)
+    if ((rc = check_block_weights(&blocks[b], C, tokens, tok_bytes, workspace, workspace_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const long long rows = static_cast<long long>(c.S) * c.T;
+  if ((rc = launch_special_rows(feats, tokens, static_cast<int>(rows), C * 2, shape->n_special, shape->T, true, st)))
+    return rc;
+  for (int b = 0; b < n_blocks; ++b)
+    if ((rc = run_block(VGGT_ATTN_GLOBAL, &c, tokens, &blocks[b], norm_eps, workspace, b == 0, st))) return rc;
+  return VGGT_ATTN_OK;
+}
