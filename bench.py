@@ -384,9 +384,10 @@ def run_ours(args):
     if not args.no_blocks:
         blocks = block_timings(V, device, stream)
         blocks["transformer"] = transformer_timings(V, device, stream)
-    sga = {}
+    sga, sharded = {}, {}
     if not args.no_modes:
         sga = sga_timings(V, device, stream, qkv, prm, out, ms / args.steps)
+        sharded = sharded_timings(V, device, stream, qkv, prm, ms / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -406,7 +407,7 @@ def run_ours(args):
                 "parallelism": f"independent replicas x{world} (weak)"}),
             "pct_of_peak": 100.0 * value / world / peak,
             "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
-            "blocks": blocks, "sga": sga, "cpu_baseline": cpu}
+            "blocks": blocks, "sga": sga, "sharded_global": sharded, "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -452,6 +453,40 @@ def sga_timings(V, device, stream, qkv, prm, out, global_ms):
         res[f"grid_{s_}x{s_}"] = {"ms": t, "kept_keys": nk, "speedup_vs_global": global_ms / t,
                                  "tflops_over_kept_keys": 4.0 * n * nk * 64 * shape.H / (t / 1000) / 1e12}
         del ws
+    return res
+
+
+def sharded_timings(V, device, stream, qkv, prm, global_ms):
+    """Query-sharded global attention on the headline workload, one rank's work for world sizes 1-8 on this
+    GPU: the rank's prologue over its S/world frames and its core over all keys (the all-gather between
+    them is not timed: one GPU here); the keys come from the whole scene's gathered buffer, filled once."""
+    import torch
+    w = W.workload(HEADLINE)
+    res = {}
+    for world in (1, 2, 4, 5):                     # divisors of the 100 frames
+        local = dataclasses.replace(w.shape, S=w.shape.S // world)
+        ws = torch.empty(V.vggt_attn_shard_workspace_size(local, world), dtype=torch.uint8, device=device)
+        qkv_r = qkv[:local.S]
+        out_r = torch.empty((local.S, local.T, local.H, 64), dtype=torch.bfloat16, device=device)
+        pro = lambda: V.vggt_attn_global_shard_prologue(local, world, qkv_r, prm["q_gamma"], prm["q_beta"],  # noqa: E731
+                                                       prm["k_gamma"], prm["k_beta"], ws, None, stream)
+        core = lambda: V.vggt_attn_global_shard_core(local, world, out_r, ws, None, stream)  # noqa: E731
+        pro()
+        k_send, v_send, k_all, v_all = V.vggt_attn_shard_buffers(local, world, ws)
+        for r in range(world):                     # stand-in for the all-gather: the rank's block, repeated
+            k_all[r * k_send.shape[0]:(r + 1) * k_send.shape[0]].copy_(k_send)
+            v_all[r * v_send.shape[0]:(r + 1) * v_send.shape[0]].copy_(v_send)
+        core()
+        t_pro = cuda_time_ms(pro, stream, 3)
+        t_core = cuda_time_ms(core, stream, 3)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        gather_bytes = 2 * (world - 1) * k_send.numel() * 2          # k and v blocks received per rank
+        res[f"world_{world}"] = {"rank_prologue_ms": t_pro, "rank_core_ms": t_core,
+                                 "rank_compute_ms": t_pro + t_core,
+                                 "speedup_vs_1gpu_global": global_ms / (t_pro + t_core),
+                                 "allgather_bytes_per_rank": gather_bytes,
+                                 "allgather_ms_at_770GBs": gather_bytes / 770e9 * 1e3}
+        del ws, out_r
     return res
 
 

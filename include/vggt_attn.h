@@ -334,6 +334,43 @@ int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_bl
                             void* cuda_stream);
 
 /* ------------------------------------------------------------------------
+ * Query-sharded global attention over `world` ranks (one GPU each).  Rank r
+ * holds frames [r S, (r+1) S) of the scene, S = shape->S (the LOCAL frame
+ * count; every rank the same): its queries attend to the keys of all world S
+ * frames.  The exchange step is an all-gather of the normalised, rotated keys
+ * and of the values; everything else is local.  Three calls per rank:
+ *
+ *   1. vggt_attn_global_shard_prologue: the global-mode prologue on the
+ *      rank's qkv (bf16 [S][T][3][H][64]): q into the workspace's q plane,
+ *      k (QK-LayerNorm + RoPE) and a copy of v token-major into the send
+ *      buffers k_send, v_send (bf16 [S T][H][64] each).
+ *   2. the caller all-gathers k_send -> k_all and v_send -> v_all (bf16
+ *      [world S T][H][64], rank-major: rank r's block at token offset r S T),
+ *      e.g. NCCL all-gather over NVLink; vggt_attn_shard_buffers gives the
+ *      four buffers' addresses inside the workspace.
+ *   3. vggt_attn_global_shard_core: the attention core of the rank's S T
+ *      queries over all world S T keys into out (bf16 [S][T][H][64]).
+ *
+ * RoPE positions are per frame as in global mode, so the result equals rows
+ * [r S T, (r+1) S T) of vggt_attn_global on the whole scene (bit for bit:
+ * every query row sees the same keys in the same 64-key steps).  world = 1
+ * is plain global attention with the copies in between.  The workspace
+ * (vggt_attn_shard_workspace_size bytes) holds the status word, the q plane,
+ * both send buffers and both gathered buffers; the first kernel of call 1
+ * clears the status word.  Calls are asynchronous on cuda_stream, validate
+ * every argument before enqueueing anything and allocate nothing;
+ * vggt_attn_shard_buffers does no device work. */
+size_t vggt_attn_shard_workspace_size(const vggt_attn_shape* shape, int world);
+int vggt_attn_shard_buffers(const vggt_attn_shape* shape, int world, void* workspace, void** k_send,
+                            void** v_send, void** k_all, void** v_all);
+int vggt_attn_global_shard_prologue(const vggt_attn_shape* shape, int world, const void* qkv,
+                                    const float* q_gamma, const float* q_beta,
+                                    const float* k_gamma, const float* k_beta,
+                                    void* workspace, size_t workspace_bytes, void* cuda_stream);
+int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int world, void* out,
+                                void* workspace, size_t workspace_bytes, void* cuda_stream);
+
+/* ------------------------------------------------------------------------
  * Camera-head trunk (VGGT-Omega Aggregator explainer, section 4: the camera
  * head takes the first 17 tokens of every frame -- camera and register
  * tokens -- from the last layer's features and mixes them across frames once

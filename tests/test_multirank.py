@@ -56,3 +56,39 @@ def test_single_process_defaults():
     assert bench.dist_env()[:2] == (0, 1)
     assert bench.reduce_max(3.5) == 3.5
     assert bench.shard_plan(1, 0, 1003)["seed"] == 1003
+
+
+def _gather_worker(rank, world, port, results):
+    import datetime
+    import sys
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    from vit_attention_b200.sharded import gather_kv
+    L, H = 5, 2
+    k_send = torch.full((L, H, 64), float(rank + 1))
+    v_send = -k_send - 0.5
+    k_all = torch.empty((world * L, H, 64))
+    v_all = torch.empty((world * L, H, 64))
+    gather_kv(k_send, v_send, k_all, v_all)
+    results[rank] = (k_all[:, 1, 63].tolist(), v_all[:, 0, 0].tolist())
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sharded_global_gathers_kv_in_rank_order():
+    """The exchange step of query-sharded global attention: every rank ends with
+    all ranks' key/value rows, rank r's block at token offset r * L."""
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        results = m.dict()
+        mp.spawn(_gather_worker, args=(world, port, results), nprocs=world, join=True)
+        res = dict(results)
+    for r in range(world):
+        k, v = res[r]
+        assert k == [1.0] * 5 + [2.0] * 5
+        assert v == [-1.5] * 5 + [-2.5] * 5

@@ -83,6 +83,11 @@ _SIGNATURES = {
     "vggt_aggregator_forward": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
                                        ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int), _int,
                                        ctypes.c_float, _vp, _sz, _vp]),
+    "vggt_attn_shard_workspace_size": (_sz, [_shape_p, _int]),
+    "vggt_attn_shard_buffers": (_int, [_shape_p, _int, _vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
+                                       ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
+    "vggt_attn_global_shard_prologue": (_int, [_shape_p, _int, _vp, _fp, _fp, _fp, _fp, _vp, _sz, _vp]),
+    "vggt_attn_global_shard_core": (_int, [_shape_p, _int, _vp, _vp, _sz, _vp]),
     "vggt_camera_trunk_workspace_size": (_sz, [_shape_p]),
     "vggt_camera_trunk_forward": (_int, [_shape_p, _vp, _vp, ctypes.POINTER(vggt_block_weights), _int,
                                          ctypes.c_float, _vp, _sz, _vp]),
@@ -312,3 +317,38 @@ def vggt_camera_trunk_forward(shape, feats, tokens, blocks, norm_eps, workspace,
                                         norm_eps, _ptr(workspace), _nbytes(workspace, workspace_bytes),
                                         _stream(stream))
     _check(rc, "vggt_camera_trunk_forward")
+
+
+def vggt_attn_shard_workspace_size(shape, world: int) -> int:
+    return _lib.vggt_attn_shard_workspace_size(ctypes.byref(make_shape(shape)), world)
+
+
+def vggt_attn_shard_buffers(shape, world: int, workspace):
+    """Views (bf16 tensors) of the send and gathered k/v buffers inside a uint8 workspace tensor:
+    (k_send, v_send, k_all, v_all), shapes [S*T, H, 64] and [world*S*T, H, 64]."""
+    import torch
+    ptrs = [ctypes.c_void_p() for _ in range(4)]
+    rc = _lib.vggt_attn_shard_buffers(ctypes.byref(make_shape(shape)), world, _ptr(workspace),
+                                      *[ctypes.byref(p) for p in ptrs])
+    _check(rc, "vggt_attn_shard_buffers")
+    n = shape.S * shape.T
+    views = []
+    for p, rows in zip(ptrs, (n, n, world * n, world * n)):
+        off = p.value - workspace.data_ptr()
+        nbytes = rows * shape.H * 64 * 2
+        views.append(workspace[off:off + nbytes].view(torch.bfloat16).view(rows, shape.H, 64))
+    return tuple(views)
+
+
+def vggt_attn_global_shard_prologue(shape, world, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace,
+                                    workspace_bytes=None, stream=None):
+    rc = _lib.vggt_attn_global_shard_prologue(ctypes.byref(make_shape(shape)), world, _ptr(qkv), _ptr(q_gamma),
+                                              _ptr(q_beta), _ptr(k_gamma), _ptr(k_beta), _ptr(workspace),
+                                              _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_global_shard_prologue")
+
+
+def vggt_attn_global_shard_core(shape, world, out, workspace, workspace_bytes=None, stream=None):
+    rc = _lib.vggt_attn_global_shard_core(ctypes.byref(make_shape(shape)), world, _ptr(out), _ptr(workspace),
+                                          _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_global_shard_core")

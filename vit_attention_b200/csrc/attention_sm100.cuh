@@ -114,10 +114,13 @@ constexpr uint32_t POLY_PAIR_MASK = 0x80u;
 // shape instead (attention_frame_persistent.cuh): its CTAs take tile after
 // tile and start the next tile's products during the last one's epilogue,
 // 2 % faster on the 500-frame workload.
-template <int NQ_, bool SGA_ = false>
+template <int NQ_, bool SGA_ = false, bool KTM_ = false>
 struct CoreCfg {
   static constexpr int NQ = NQ_;
   static constexpr bool SGA = SGA_;   // subsampled global attention epilogue
+  // Keys token-major, [Lk][H][64] like the values (query-sharded global mode:
+  // the keys all ranks gathered), instead of one [B*Lk][64] plane per head.
+  static constexpr bool KTM = KTM_;
   static constexpr int CTAS_PER_SM = NQ_ == 2 ? 1 : 2;
   static constexpr int STAGES = NQ_ == 2 ? 8 : 5;
   static constexpr int OFF_Q = 0;                                  // NQ tiles
@@ -574,7 +577,10 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * KV_BYTES);
-        tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
+        if constexpr (C::KTM)
+          tma_load_4d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+        else
+          tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
         tma_load_4d(sbase + OFF_V + st * KV_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
         ++issued[st];
       }

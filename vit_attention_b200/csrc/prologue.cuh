@@ -62,14 +62,15 @@ struct PrologueParams {
   const float* gamma[2];  // q, k
   const float* beta[2];
   uint16_t* ws_qk[2];     // q, k destinations
-  uint16_t* ws_v;         // register mode only
+  uint16_t* ws_v;         // v copied token-major [L][H][64] when n_c == 3
+  int k_token_major;      // k written token-major [L][H][64] (like v) instead of the head planes
   int* status;         // cleared by block 0 when zero_status (the first kernel of a call)
   int zero_status;
   int n_tok;              // tokens in the mode's token list (< 2^31, checked on the host)
   int T, H, n_special, grid_h, grid_w;
   int mode;               // VGGT_ATTN_FRAME / GLOBAL / REGISTER
   int L;                  // tokens per problem in the workspace
-  int n_c;                // 2 (q, k) or 3 (q, k, v in register mode)
+  int n_c;                // 2 (q, k) or 3 (q, k and a copy of v: register mode, sharded global mode)
   FastDiv div_nspec, div_L, div_T, div_gw;
   float eps;
   float q_mult;           // softmax_scale * log2(e)
@@ -230,7 +231,8 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
         ob.y = pack_bf16x2(xb[2] * mult, xb[3] * mult);
         ob.z = pack_bf16x2(xb[4] * mult, xb[5] * mult);
         ob.w = pack_bf16x2(xb[6] * mult, xb[7] * mult);
-        uint16_t* dst = p.ws_qk[c] + w[k].dst_qk + row_dst;
+        uint16_t* dst = (c == 1 && p.k_token_major) ? p.ws_qk[1] + w[k].dst_v + h * 64 + base
+                                                    : p.ws_qk[c] + w[k].dst_qk + row_dst;
         *reinterpret_cast<uint4*>(dst) = oa;
         *reinterpret_cast<uint4*>(dst + 16) = ob;
       }

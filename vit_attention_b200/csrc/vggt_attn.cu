@@ -134,10 +134,12 @@ bool make_map(CUtensorMap* map, const void* base, int rank, const cuuint64_t* di
 
 // clear_status: the prologue is the call's first kernel (the attention entry
 // points); inside a block an earlier kernel has cleared the status word and
-// may already have recorded an error in it.
+// may already have recorded an error in it.  shard_k / shard_v (global mode,
+// one rank's frames): k and a copy of v go token-major ([L][H][64]) to these
+// buffers, the ones all ranks gather, instead of k to the workspace plane.
 int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const float* gq, const float* bq,
                     const float* gk, const float* bk, const WorkspaceView& w, cudaStream_t stream,
-                    bool clear_status = true) {
+                    bool clear_status = true, uint16_t* shard_k = nullptr, uint16_t* shard_v = nullptr) {
   const ModeGeometry g = geometry(s, mode);
   vggt::PrologueParams p;
   p.qkv = static_cast<const uint16_t*>(qkv);
@@ -148,6 +150,14 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.ws_qk[0] = w.q;
   p.ws_qk[1] = w.k;
   p.ws_v = w.v;
+  p.k_token_major = 0;
+  p.n_c = g.n_c;
+  if (shard_k) {
+    p.ws_qk[1] = shard_k;
+    p.ws_v = shard_v;
+    p.k_token_major = 1;
+    p.n_c = 3;
+  }
   p.status = w.status;
   p.zero_status = clear_status ? 1 : 0;
   p.n_tok = static_cast<int>(g.n_tok);
@@ -158,7 +168,6 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   p.grid_w = s->grid_w;
   p.mode = mode;
   p.L = static_cast<int>(g.L);
-  p.n_c = g.n_c;
   p.div_nspec = vggt::make_fastdiv(static_cast<uint32_t>(s->n_special));
   p.div_L = vggt::make_fastdiv(static_cast<uint32_t>(g.L));
   p.div_T = vggt::make_fastdiv(static_cast<uint32_t>(s->T));
@@ -171,7 +180,7 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   // One 4-lane group per head row of a token (a group loops over rows when a
   // token has more than 64); as many blocks as fit on the device at once,
   // each striding over the tokens four at a time.
-  const int ch = g.n_c * s->H;
+  const int ch = p.n_c * s->H;
   const int threads = ch <= 64 ? 4 * ch : 256;
   const size_t smem = static_cast<size_t>(s->grid_h + s->grid_w) * 16 * sizeof(float2);
   if (smem > 48 * 1024 &&
@@ -1133,4 +1142,145 @@ extern "C" int vggt_camera_trunk_forward(const vggt_attn_shape* shape, const voi
   for (int b = 0; b < n_blocks; ++b)
     if ((rc = run_block(VGGT_ATTN_GLOBAL, &c, tokens, &blocks[b], norm_eps, workspace, b == 0, st))) return rc;
   return VGGT_ATTN_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Query-sharded global attention: local prologue, all-gather of k and v by
+// the caller, core over all ranks' keys.
+namespace {
+
+constexpr int kMaxShardWorld = 1024;
+
+struct ShardLayout {
+  WorkspaceView w;          // status, q plane [H][L][64] (k plane unused)
+  uint16_t* k_send;         // [L][H][64]
+  uint16_t* v_send;
+  uint16_t* k_all;          // [world L][H][64]
+  uint16_t* v_all;
+  long long L, Lk;
+  size_t bytes;
+};
+
+ShardLayout shard_layout(const vggt_attn_shape* s, int world, void* ws) {
+  ShardLayout S{};
+  S.L = static_cast<long long>(s->S) * s->T;
+  S.Lk = S.L * world;
+  const size_t row = static_cast<size_t>(s->H) * 64 * 2;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  S.w.status = reinterpret_cast<int*>(base);
+  size_t off = kStatusBytes;
+  S.w.q = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(S.L * row);
+  S.w.k = nullptr;
+  S.w.v = nullptr;
+  S.k_send = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(S.L * row);
+  S.v_send = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(S.L * row);
+  S.k_all = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(S.Lk * row);
+  S.v_all = reinterpret_cast<uint16_t*>(base + off);
+  off += align256(S.Lk * row);
+  S.w.bytes = off;
+  S.bytes = off;
+  return S;
+}
+
+int check_shard_shape(const vggt_attn_shape* s, int world) {
+  if (world < 1 || world > kMaxShardWorld) return VGGT_ATTN_ERR_INVALID_ARG;
+  int rc = check_shape(s, VGGT_ATTN_GLOBAL);
+  if (rc) return rc;
+  vggt_attn_shape whole = *s;
+  const long long S = static_cast<long long>(s->S) * world;
+  if (S > INT32_MAX) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  whole.S = static_cast<int>(S);
+  return check_shape(&whole, VGGT_ATTN_GLOBAL);   // token counts of the whole scene
+}
+
+int check_shard_ws(const vggt_attn_shape* s, int world, void* ws, size_t ws_bytes) {
+  if (!ws) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(ws, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  if (ws_bytes < shard_layout(s, world, nullptr).bytes) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  return VGGT_ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" size_t vggt_attn_shard_workspace_size(const vggt_attn_shape* shape, int world) {
+  if (check_shard_shape(shape, world) != VGGT_ATTN_OK) return 0;
+  return shard_layout(shape, world, nullptr).bytes;
+}
+
+extern "C" int vggt_attn_shard_buffers(const vggt_attn_shape* shape, int world, void* workspace, void** k_send,
+                                       void** v_send, void** k_all, void** v_all) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if (!workspace || !k_send || !v_send || !k_all || !v_all) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256)) return VGGT_ATTN_ERR_MISALIGNED;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  *k_send = L.k_send;
+  *v_send = L.v_send;
+  *k_all = L.k_all;
+  *v_all = L.v_all;
+  return VGGT_ATTN_OK;
+}
+
+extern "C" int vggt_attn_global_shard_prologue(const vggt_attn_shape* shape, int world, const void* qkv,
+                                               const float* q_gamma, const float* q_beta, const float* k_gamma,
+                                               const float* k_beta, void* workspace, size_t workspace_bytes,
+                                               void* cuda_stream) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes))) return rc;
+  if (!qkv || !q_gamma || !q_beta || !k_gamma || !k_beta) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(qkv, 16) || !aligned(q_gamma, 16) || !aligned(q_beta, 16) || !aligned(k_gamma, 16) ||
+      !aligned(k_beta, 16))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t qkv_bytes = static_cast<size_t>(shape->S) * shape->T * 3 * shape->H * 128;
+  if (overlaps(qkv, qkv_bytes, workspace, workspace_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  return launch_prologue(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, L.w,
+                         static_cast<cudaStream_t>(cuda_stream), true, L.k_send, L.v_send);
+}
+
+extern "C" int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int world, void* out, void* workspace,
+                                           size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes))) return rc;
+  if (!out) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t out_bytes = static_cast<size_t>(shape->S) * shape->T * shape->H * 128;
+  if (overlaps(out, out_bytes, workspace, workspace_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  const long long H = shape->H;
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(L.L), static_cast<cuuint64_t>(H)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(L.L) * 128};
+    const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};
+    if (!make_map(&mq, L.w.q, 3, dims, strides, box_q)) return VGGT_ATTN_ERR_CUDA;
+  }
+  {
+    // gathered keys and values, [Lk][H][64]: (dim, head, token, 1)
+    const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L.Lk), 1};
+    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(L.Lk) * H * 128};
+    const cuuint32_t box[4] = {64, 1, vggt::core::BN, 1};
+    if (!make_map(&mk, L.k_all, 4, dims, strides, box) || !make_map(&mv, L.v_all, 4, dims, strides, box))
+      return VGGT_ATTN_ERR_CUDA;
+  }
+  vggt::CoreParams p{};
+  p.L = static_cast<int>(L.L);
+  p.Lk = static_cast<int>(L.Lk);
+  p.H = shape->H;
+  p.B = 1;
+  p.out_T = shape->T;
+  p.out_group = static_cast<int>(L.L);
+  p.out = static_cast<uint16_t*>(out);
+  p.status = L.w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  ModeGeometry g{1, L.L, L.L, 2};
+  return launch_core_cfg<vggt::CoreCfg<2, false, true>>(g, shape->H, mq, mk, mv, p, static_cast<cudaStream_t>(cuda_stream));
 }
