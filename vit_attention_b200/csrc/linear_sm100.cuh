@@ -33,6 +33,11 @@
 //                (qkv epilogue: normalises and rotates), and writes its 128-byte
 //                row of the chunk into the staging buffer; one thread stores
 //                the chunk with TMA.
+//   warps 8-11   (gelu and resid epilogues only, 384 threads) a second
+//                epilogue warpgroup: warps 4-7 take chunks 0-1 of every tile,
+//                warps 8-11 chunks 2-3, each with its own staging buffer, so
+//                that the heavier per-element work keeps up with the products
+//                (5 % off a frame-mode transformer block).
 // Every mbarrier wait is bounded (wait_bounded); on expiry the CTA records
 // VGGT_ATTN_ERR_TIMEOUT in the status word and drains what it has in flight.
 #pragma once
@@ -45,6 +50,7 @@ namespace vggt {
 
 namespace lin {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+enum { EPI_STD = 0, EPI_GELU = 1, EPI_RESID = 2 };     // EPI_STD: plain or qkv (LinearParams::fused)
 constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
 constexpr int OFF_A = 0;
@@ -58,16 +64,24 @@ enum {
   BAR_ACC_EMPTY = BAR_ACC_FULL + 2,    // [accumulator]
   BAR_STAGE_FULL = BAR_ACC_EMPTY + 2,  // every epilogue thread wrote its row of the chunk
   BAR_STAGE_FREE = BAR_STAGE_FULL + 1, // the chunk's TMA store has read the buffer
-  BAR_DRAIN = BAR_STAGE_FREE + 1,
+  BAR_STAGE_FULL2 = BAR_STAGE_FREE + 1, // the same for the second epilogue warpgroup's buffer
+  BAR_STAGE_FREE2 = BAR_STAGE_FULL2 + 1,
+  BAR_DRAIN = BAR_STAGE_FREE2 + 1,
   N_BARS = BAR_DRAIN + 1
 };
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
 constexpr int OFF_ROPE = OFF_MISC + 16;                // cos/sin table (qkv epilogue)
 constexpr int THREADS = 256;
+// The GELU and residual epilogues do more per element: they run on two
+// warpgroups (warps 4-7 take the tile's first two 64-column chunks, warps
+// 8-11 the last two), each with its own staging buffer; the second buffer
+// sits where the qkv epilogue keeps its RoPE table.
+constexpr int OFF_STAGE2 = (OFF_ROPE + 1023) & ~1023;
+__host__ __device__ constexpr int epi_warpgroups(int epi) { return epi == EPI_STD ? 1 : 2; }
+__host__ __device__ constexpr int threads_for(int epi) { return 128 * (1 + epi_warpgroups(epi)); }
 constexpr uint32_t TMEM_COLS = 512;                    // two 256-column accumulators
 constexpr uint32_t IDESC = idesc_bf16_f32(BM, BN, 0, 0);
 constexpr int REGS_AT_LAUNCH = 168;
-enum { EPI_STD = 0, EPI_GELU = 1, EPI_RESID = 2 };     // EPI_STD: plain or qkv (LinearParams::fused)
 }  // namespace lin
 
 struct LinearParams {
@@ -104,7 +118,8 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-__host__ __device__ inline int linear_smem_bytes(int grid_h, int grid_w) {
+__host__ __device__ constexpr int linear_smem_bytes(int grid_h, int grid_w, int epi = lin::EPI_STD) {
+  if (epi != lin::EPI_STD) return lin::OFF_STAGE2 + lin::BM * 128 + 1024;
   return lin::OFF_ROPE + (grid_h + grid_w) * 16 * 8 + 1024;   // + slack to align the base to 1024 B
 }
 
@@ -138,12 +153,31 @@ template <int EPI>
 __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t acc, int m0, int n0, int row,
                                                 bool leader, uint8_t* stage, uint32_t bar0, volatile int* abort_flag,
                                                 int& chunk, const CUtensorMap* to0, const CUtensorMap* to1,
-                                                const CUtensorMap* to2, const float2* rope_tab) {
+                                                const CUtensorMap* to2, const float2* rope_tab, int ck_begin,
+                                                int ck_end, int bar_full, int bar_free) {
   using namespace lin;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int m = m0 + row;                 // rows past M compute garbage that TMA clips
+  // Residual epilogue: the residual of the next chunk is loaded while this
+  // one is converted (rows past M have none).
+  uint4 rnext[8];
+  if constexpr (EPI == lin::EPI_RESID) {
+    const uint4* rrow = reinterpret_cast<const uint4*>(p.resid + static_cast<long long>(m) * p.N + n0 + ck_begin * 64);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) rnext[k] = m < p.M ? rrow[k] : make_uint4(0u, 0u, 0u, 0u);
+  }
 #pragma unroll 1
-  for (int ck = 0; ck < BN / 64; ++ck, ++chunk) {
+  for (int ck = ck_begin; ck < ck_end; ++ck, ++chunk) {
+    uint4 rcur[8];
+    if constexpr (EPI == lin::EPI_RESID) {
+#pragma unroll
+      for (int k = 0; k < 8; ++k) rcur[k] = rnext[k];
+      if (ck + 1 < ck_end) {
+        const uint4* rrow = reinterpret_cast<const uint4*>(p.resid + static_cast<long long>(m) * p.N + n0 + (ck + 1) * 64);
+#pragma unroll
+        for (int k = 0; k < 8; ++k) rnext[k] = m < p.M ? rrow[k] : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
     uint32_t v[64];
     tmem_ld64(acc + ck * 64, v);
     tmem_wait_ld();
@@ -166,11 +200,9 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
       }
     }
     if constexpr (EPI == lin::EPI_RESID) {
-      // Rows past M have no residual (their values are clipped by the store).
-      const uint4* rrow = reinterpret_cast<const uint4*>(p.resid + static_cast<long long>(m) * p.N + col0);
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
-        const uint4 r = m < p.M ? rrow[k] : make_uint4(0u, 0u, 0u, 0u);
+        const uint4 r = rcur[k];
         const float4 l0 = __ldg(reinterpret_cast<const float4*>(p.ls + col0 + 8 * k));
         const float4 l1 = __ldg(reinterpret_cast<const float4*>(p.ls + col0 + 8 * k + 4));
         const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
@@ -184,7 +216,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
       }
     }
     const int c = (EPI == lin::EPI_STD && p.fused) ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
-    const int h = (col0 / 64) % p.H;
+    const int h = (EPI == lin::EPI_STD && p.fused) ? (col0 / 64) % p.H : 0;   // plain GEMMs have H = 0
     uint4 o[8];
     if (c == 2) {
 #pragma unroll
@@ -266,19 +298,19 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
     if (chunk > 0) {
       if (leader) {
         bulk_wait_read_all();
-        mbar_arrive(bar(BAR_STAGE_FREE));
+        mbar_arrive(bar(bar_free));
       }
-      bool ok = wait_bounded(bar(BAR_STAGE_FREE), (chunk - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x540u);
+      bool ok = wait_bounded(bar(bar_free), (chunk - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x540u);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) return false;
     }
 #pragma unroll
     for (int k = 0; k < 8; ++k) *reinterpret_cast<uint4*>(stage + row * 128 + ((k ^ (row & 7)) * 16)) = o[k];
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-    mbar_arrive(bar(BAR_STAGE_FULL));
+    mbar_arrive(bar(bar_full));
     bool ok = true;
     if (leader) {
-      ok = wait_bounded(bar(BAR_STAGE_FULL), chunk & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
+      ok = wait_bounded(bar(bar_full), chunk & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
       if (ok) {
         const uint32_t src = smem_addr(stage);
         if (EPI != lin::EPI_STD || !p.fused)
@@ -297,7 +329,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
 }
 
 template <int EPI>
-__global__ void __launch_bounds__(lin::THREADS, 1)
+__global__ void __launch_bounds__(lin::threads_for(EPI), 1)
     linear_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_w,
                   const __grid_constant__ CUtensorMap tmap_o0, const __grid_constant__ CUtensorMap tmap_o1,
                   const __grid_constant__ CUtensorMap tmap_o2, const LinearParams p) {
@@ -322,10 +354,12 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(bar(BAR_ACC_FULL + a), 1);
-      mbar_init(bar(BAR_ACC_EMPTY + a), 128);
+      mbar_init(bar(BAR_ACC_EMPTY + a), 128 * epi_warpgroups(EPI));
     }
     mbar_init(bar(BAR_STAGE_FULL), 128);
     mbar_init(bar(BAR_STAGE_FREE), 1);
+    mbar_init(bar(BAR_STAGE_FULL2), 128);
+    mbar_init(bar(BAR_STAGE_FREE2), 1);
     mbar_init(bar(BAR_DRAIN), 1);
     fence_mbar_init();
     *abort_flag = 0;
@@ -428,7 +462,10 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
     if (!skip) {
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
-      const bool leader = threadIdx.x == 128;
+      const int wg = (warp - 4) >> 2;                        // epilogue warpgroup
+      constexpr int CPW = (BN / 64) / epi_warpgroups(EPI);   // chunks per warpgroup
+      const bool leader = (threadIdx.x & 127) == 0;
+      uint8_t* stage = smem + (wg == 0 ? OFF_STAGE : OFF_STAGE2);
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       int lt = 0, chunk = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {
@@ -439,8 +476,10 @@ __global__ void __launch_bounds__(lin::THREADS, 1)
         if (!ok) break;
         tc_fence_after();
         const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
-        ok = linear_epilogue<EPI>(p, tmem + lane_base + ab * BN, m0, n0, row, leader, smem + OFF_STAGE, bar0, abort_flag,
-                             chunk, &tmap_o0, &tmap_o1, &tmap_o2, rope_tab);
+        ok = linear_epilogue<EPI>(p, tmem + lane_base + ab * BN, m0, n0, row, leader, stage, bar0, abort_flag, chunk,
+                                  &tmap_o0, &tmap_o1, &tmap_o2, rope_tab, wg * CPW, (wg + 1) * CPW,
+                                  wg == 0 ? BAR_STAGE_FULL : BAR_STAGE_FULL2,
+                                  wg == 0 ? BAR_STAGE_FREE : BAR_STAGE_FREE2);
         tc_fence_before();
         mbar_arrive(bar(BAR_ACC_EMPTY + ab));
         if (!ok) break;

@@ -505,9 +505,11 @@ int check_linear_dims(long long M, long long N, long long K) {
 template <int EPI>
 int launch_linear_epi(const vggt::LinearParams& p, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& o0,
                       const CUtensorMap& o1, const CUtensorMap& o2, int smem, unsigned grid, cudaStream_t stream) {
+  static_assert(vggt::linear_smem_bytes(0, 0, vggt::lin::EPI_GELU) <= 227 * 1024, "two staging buffers fit");
+  if (EPI != vggt::lin::EPI_STD) smem = vggt::linear_smem_bytes(0, 0, EPI);
   if (cudaFuncSetAttribute(vggt::linear_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
-  vggt::linear_kernel<EPI><<<grid, vggt::lin::THREADS, smem, stream>>>(mx, mw, o0, o1, o2, p);
+  vggt::linear_kernel<EPI><<<grid, vggt::lin::threads_for(EPI), smem, stream>>>(mx, mw, o0, o1, o2, p);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
