@@ -334,6 +334,29 @@ int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_bl
                             void* cuda_stream);
 
 /* ------------------------------------------------------------------------
+ * Host-memory pipeline: n_items independent calls of one mode (frame, global
+ * or register; one scene each, all of `shape`) whose qkv inputs and outputs
+ * live in pinned host memory.  Item i's qkv (h_qkv[i], bf16
+ * [S][T][3][H][64]) is copied to the device on h2d_stream, attended on
+ * compute_stream (prologue + core, as vggt_attn_frame/global/register) and
+ * its result copied back to h_out[i] (bf16 [S][T][H][64]) on d2h_stream;
+ * two device staging sets in the workspace let the copies of items i+1 and
+ * i-1 run during item i's kernels.  In register mode only the special-token
+ * rows of h_out[i] are written (one strided copy).  q/k gamma/beta are
+ * device pointers shared by all items.  The host buffers must be page-locked
+ * (cudaHostAlloc / cudaHostRegister; VGGT_ATTN_ERR_INVALID_ARG otherwise)
+ * and stay valid until d2h_stream has completed; the call returns after
+ * enqueueing (the three streams may be the same stream, which serialises the
+ * items).  The first kernel clears the workspace status word.  Workspace:
+ * vggt_attn_host_pipeline_workspace_size(shape, mode) bytes. */
+size_t vggt_attn_host_pipeline_workspace_size(const vggt_attn_shape* shape, int mode);
+int vggt_attn_host_pipeline(int mode, const vggt_attn_shape* shape, int n_items, const void* const* h_qkv,
+                            const float* q_gamma, const float* q_beta,
+                            const float* k_gamma, const float* k_beta, void* const* h_out,
+                            void* workspace, size_t workspace_bytes,
+                            void* compute_stream, void* h2d_stream, void* d2h_stream);
+
+/* ------------------------------------------------------------------------
  * Query-sharded global attention over `world` ranks (one GPU each).  Rank r
  * holds frames [r S, (r+1) S) of the scene, S = shape->S (the LOCAL frame
  * count; every rank the same): its queries attend to the keys of all world S

@@ -83,6 +83,9 @@ _SIGNATURES = {
     "vggt_aggregator_forward": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
                                        ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int), _int,
                                        ctypes.c_float, _vp, _sz, _vp]),
+    "vggt_attn_host_pipeline_workspace_size": (_sz, [_shape_p, _int]),
+    "vggt_attn_host_pipeline": (_int, [_int, _shape_p, _int, ctypes.POINTER(_vp), _fp, _fp, _fp, _fp,
+                                       ctypes.POINTER(_vp), _vp, _sz, _vp, _vp, _vp]),
     "vggt_attn_shard_workspace_size": (_sz, [_shape_p, _int]),
     "vggt_attn_shard_buffers": (_int, [_shape_p, _int, _vp, ctypes.POINTER(_vp), ctypes.POINTER(_vp),
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
@@ -352,3 +355,28 @@ def vggt_attn_global_shard_core(shape, world, out, workspace, workspace_bytes=No
     rc = _lib.vggt_attn_global_shard_core(ctypes.byref(make_shape(shape)), world, _ptr(out), _ptr(workspace),
                                           _nbytes(workspace, workspace_bytes), _stream(stream))
     _check(rc, "vggt_attn_global_shard_core")
+
+
+def vggt_attn_host_pipeline_workspace_size(shape, mode) -> int:
+    mode = MODES.get(mode, mode)
+    return _lib.vggt_attn_host_pipeline_workspace_size(ctypes.byref(make_shape(shape)), mode)
+
+
+def vggt_attn_host_pipeline(mode, shape, h_qkv, q_gamma, q_beta, k_gamma, k_beta, h_out, workspace,
+                            workspace_bytes=None, compute_stream=None, h2d_stream=None, d2h_stream=None):
+    """Attend len(h_qkv) scenes whose qkv inputs and outputs are pinned host tensors; the copies of
+    neighbouring scenes run on h2d_stream / d2h_stream during each scene's kernels on compute_stream.
+    Returns after enqueueing: synchronise d2h_stream before reading h_out."""
+    mode = MODES.get(mode, mode)
+    n = len(h_qkv)
+    if len(h_out) != n:
+        raise ValueError("one output buffer per input")
+    qs = (_vp * max(n, 1))(*[_ptr(t) for t in h_qkv])
+    outs = (_vp * max(n, 1))(*[_ptr(t) for t in h_out])
+    sc = _stream(compute_stream)
+    rc = _lib.vggt_attn_host_pipeline(mode, ctypes.byref(make_shape(shape)), n, qs, _ptr(q_gamma), _ptr(q_beta),
+                                      _ptr(k_gamma), _ptr(k_beta), outs, _ptr(workspace),
+                                      _nbytes(workspace, workspace_bytes), sc,
+                                      sc if h2d_stream is None else _stream(h2d_stream),
+                                      sc if d2h_stream is None else _stream(d2h_stream))
+    _check(rc, "vggt_attn_host_pipeline")

@@ -1286,3 +1286,105 @@ extern "C" int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int wor
   ModeGeometry g{1, L.L, L.L, 2};
   return launch_core_cfg<vggt::CoreCfg<2, false, true>>(g, shape->H, mq, mk, mv, p, static_cast<cudaStream_t>(cuda_stream));
 }
+
+// ---------------------------------------------------------------------------
+// Host-memory pipeline: copies of neighbouring items overlap each item's kernels.
+namespace {
+
+struct PipeLayout {
+  size_t att_bytes, qkv_bytes, out_bytes, bytes;
+  uint8_t* qkv[2];
+  uint8_t* out[2];
+};
+
+PipeLayout pipe_layout(const vggt_attn_shape* s, int mode, void* ws) {
+  PipeLayout P{};
+  P.att_bytes = workspace_view(s, mode, nullptr).bytes;
+  P.qkv_bytes = static_cast<size_t>(s->S) * s->T * 3 * s->H * 128;
+  P.out_bytes = static_cast<size_t>(s->S) * s->T * s->H * 128;
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  size_t off = align256(P.att_bytes);
+  for (int b = 0; b < 2; ++b) {
+    P.qkv[b] = base + off;
+    off += align256(P.qkv_bytes);
+  }
+  for (int b = 0; b < 2; ++b) {
+    P.out[b] = base + off;
+    off += align256(P.out_bytes);
+  }
+  P.bytes = off;
+  return P;
+}
+
+bool pinned_host(const void* p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();   // clear the query's error state
+    return false;
+  }
+  return a.type == cudaMemoryTypeHost;
+}
+
+}  // namespace
+
+extern "C" size_t vggt_attn_host_pipeline_workspace_size(const vggt_attn_shape* shape, int mode) {
+  if (check_shape(shape, mode) != VGGT_ATTN_OK) return 0;
+  return pipe_layout(shape, mode, nullptr).bytes;
+}
+
+extern "C" int vggt_attn_host_pipeline(int mode, const vggt_attn_shape* shape, int n_items, const void* const* h_qkv,
+                                       const float* q_gamma, const float* q_beta, const float* k_gamma,
+                                       const float* k_beta, void* const* h_out, void* workspace,
+                                       size_t workspace_bytes, void* compute_stream, void* h2d_stream,
+                                       void* d2h_stream) {
+  int rc = check_shape(shape, mode);
+  if (rc) return rc;
+  if (n_items < 0 || (n_items > 0 && (!h_qkv || !h_out)) || !workspace) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!q_gamma || !q_beta || !k_gamma || !k_beta) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(workspace, 256) || !aligned(q_gamma, 16) || !aligned(q_beta, 16) || !aligned(k_gamma, 16) ||
+      !aligned(k_beta, 16))
+    return VGGT_ATTN_ERR_MISALIGNED;
+  const PipeLayout P = pipe_layout(shape, mode, workspace);
+  if (workspace_bytes < P.bytes) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  for (int i = 0; i < n_items; ++i)
+    if (!h_qkv[i] || !h_out[i]) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  for (int i = 0; i < n_items; ++i)
+    if (!pinned_host(h_qkv[i]) || !pinned_host(h_out[i])) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (n_items == 0) return VGGT_ATTN_OK;
+  cudaStream_t sc = static_cast<cudaStream_t>(compute_stream);
+  cudaStream_t si = static_cast<cudaStream_t>(h2d_stream);
+  cudaStream_t so = static_cast<cudaStream_t>(d2h_stream);
+  cudaEvent_t ev[3][2] = {};   // [h2d done, compute done, d2h done][staging set]
+  for (int k = 0; k < 3 && rc == VGGT_ATTN_OK; ++k)
+    for (int b = 0; b < 2; ++b)
+      if (cudaEventCreateWithFlags(&ev[k][b], cudaEventDisableTiming) != cudaSuccess) rc = VGGT_ATTN_ERR_CUDA;
+  const WorkspaceView w = workspace_view(shape, mode, workspace);
+  const size_t row_bytes = static_cast<size_t>(shape->H) * 128;
+  for (int i = 0; i < n_items && rc == VGGT_ATTN_OK; ++i) {
+    const int b = i & 1;
+    // H2D of item i into set b, after item i-2's kernels have read it.
+    if (i >= 2 && cudaStreamWaitEvent(si, ev[1][b], 0) != cudaSuccess) { rc = VGGT_ATTN_ERR_CUDA; break; }
+    if (cudaMemcpyAsync(P.qkv[b], h_qkv[i], P.qkv_bytes, cudaMemcpyHostToDevice, si) != cudaSuccess ||
+        cudaEventRecord(ev[0][b], si) != cudaSuccess) { rc = VGGT_ATTN_ERR_CUDA; break; }
+    // Kernels of item i, after its H2D and after item i-2's D2H has read out set b.
+    if (cudaStreamWaitEvent(sc, ev[0][b], 0) != cudaSuccess ||
+        (i >= 2 && cudaStreamWaitEvent(sc, ev[2][b], 0) != cudaSuccess)) { rc = VGGT_ATTN_ERR_CUDA; break; }
+    if ((rc = launch_prologue(mode, shape, P.qkv[b], q_gamma, q_beta, k_gamma, k_beta, w, sc, i == 0))) break;
+    if ((rc = launch_core(mode, shape, P.qkv[b], P.out[b], w, sc))) break;
+    if (cudaEventRecord(ev[1][b], sc) != cudaSuccess) { rc = VGGT_ATTN_ERR_CUDA; break; }
+    // D2H of item i (register mode: the special rows of every frame only).
+    if (cudaStreamWaitEvent(so, ev[1][b], 0) != cudaSuccess) { rc = VGGT_ATTN_ERR_CUDA; break; }
+    cudaError_t e;
+    if (mode == VGGT_ATTN_REGISTER)
+      e = cudaMemcpy2DAsync(h_out[i], shape->T * row_bytes, P.out[b], shape->T * row_bytes,
+                            shape->n_special * row_bytes, shape->S, cudaMemcpyDeviceToHost, so);
+    else
+      e = cudaMemcpyAsync(h_out[i], P.out[b], P.out_bytes, cudaMemcpyDeviceToHost, so);
+    if (e != cudaSuccess || cudaEventRecord(ev[2][b], so) != cudaSuccess) { rc = VGGT_ATTN_ERR_CUDA; break; }
+  }
+  for (int k = 0; k < 3; ++k)
+    for (int b = 0; b < 2; ++b)
+      if (ev[k][b]) cudaEventDestroy(ev[k][b]);   // released once the recorded work completes
+  return rc;
+}
