@@ -54,7 +54,9 @@ int check_shape(const vggt_attn_shape* s, int mode) {
   const long long n = static_cast<long long>(s->S) * s->T;
   if (n > (1LL << 31) - 1 - 256) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // int token indices in the core
   if (n * 3 * s->H > (1LL << 31) - 1) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // int row indices in the prologue
-  if (mode == VGGT_ATTN_FRAME && s->S > 65535) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;  // grid.z
+  if (mode == VGGT_ATTN_FRAME &&
+      (static_cast<long long>(s->T) + 127) / 128 * s->H * s->S > INT32_MAX)   // int unit indices of the frame core
+    return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
   return VGGT_ATTN_OK;
 }
 
@@ -237,8 +239,7 @@ int launch_frame_persistent(const ModeGeometry& g, int H, const CUtensorMap& mq,
     return VGGT_ATTN_ERR_CUDA;
   vggt::FrameUnits fu;
   fu.n_qt = static_cast<int>((g.L + vggt::core::BM - 1) / vggt::core::BM);
-  const long long n_units = static_cast<long long>(fu.n_qt) * H * g.B;
-  if (n_units > INT32_MAX) return VGGT_ATTN_ERR_INVALID_ARG;
+  const long long n_units = static_cast<long long>(fu.n_qt) * H * g.B;   // < 2^31: checked with the shape
   fu.n_units = static_cast<int>(n_units);
   long long grid = static_cast<long long>(sms) * vggt::fp::CTAS_PER_SM;
   if (grid > n_units) grid = n_units;
