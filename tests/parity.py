@@ -7,7 +7,7 @@ import numpy as np
 import oracle as O
 import workloads as W
 
-MAX_ABS_TOL = 2e-2     # spec tolerance against the fp64 oracle
+MAX_ABS_TOL = 2e-2     # stated parity tolerance against the fp64 oracle
 REL_FRO_TOL = 5e-3
 
 

@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
 the same seeded bf16 inputs, element by element on every compared row.
-Tolerance (the benchmark spec): max-abs <= 2e-2 and relative Frobenius <= 5e-3."""
+Tolerance (the stated parity bar): max-abs <= 2e-2 and relative Frobenius <= 5e-3."""
 import numpy as np
 import pytest
 
