@@ -60,29 +60,47 @@ def _affine(x: np.ndarray, w_bits, b) -> np.ndarray:
     return y if b is None else y + np.asarray(b, np.float64)
 
 
-def block_forward(mode: str, shape, x, w, norm_eps: float) -> np.ndarray:
+def block_forward(mode: str, shape, x, w, norm_eps: float, rows=None) -> np.ndarray:
     """One block applied to token features x (bf16 bits or fp64, ``[S*T, C]``).
 
     Returns fp64 ``[S*T, C]``.  mode: "frame", "global" or "register"; in
-    register mode only the rows of the special tokens change.
+    register mode only the rows of the special tokens change.  ``rows``
+    (flat token indices; special tokens only in register mode): return just
+    those output rows, ``[len(rows), C]`` (every token still provides keys).
     """
     x = bf16_to_f64(x) if x.dtype == np.uint16 else np.asarray(x, np.float64)
     C = shape.H * HEAD_DIM
-    rows = register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T, dtype=np.int64)
-    # Attention branch: qkv of every token (only rows in `rows` are read in
-    # register mode, whose keys and queries are the special tokens).
-    h = token_layer_norm(x, w["norm1_gamma"], w["norm1_beta"], norm_eps)
-    qkv = _affine(h, w["w_qkv"], w.get("b_qkv")).reshape(shape.S, shape.T, 3, shape.H, HEAD_DIM)
+    subset = rows is not None
+    if not subset:
+        rows = register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T, dtype=np.int64)
+    rows = np.asarray(rows, dtype=np.int64)
+    # Attention branch: qkv of the tokens the mode's attention reads (the keys
+    # of the returned rows and the rows themselves); other entries stay 0 and
+    # are never read.
+    if mode == "register":
+        need = register_tokens(shape)
+    elif mode == "frame" and subset:
+        frames = np.unique(rows // shape.T)
+        need = (frames[:, None] * shape.T + np.arange(shape.T)[None, :]).reshape(-1)
+    else:
+        need = np.arange(shape.S * shape.T, dtype=np.int64)
+    h = token_layer_norm(x[need], w["norm1_gamma"], w["norm1_beta"], norm_eps)
+    qkv = np.zeros((shape.S * shape.T, 3 * C))
+    qkv[need] = _affine(h, w["w_qkv"], w.get("b_qkv"))
+    qkv = qkv.reshape(shape.S, shape.T, 3, shape.H, HEAD_DIM)
     inputs = {"qkv_f64": qkv}
     for name in ("q_gamma", "q_beta", "k_gamma", "k_beta"):
         inputs[name] = w[name]
     a = attn_mode(mode, shape, inputs, rows).reshape(len(rows), C)
-    y = x.copy()
     xr = x[rows] + np.asarray(w["ls1"], np.float64) * _affine(a, w["w_proj"], w.get("b_proj"))
     # MLP branch on the same rows.
     h2 = token_layer_norm(xr, w["norm2_gamma"], w["norm2_beta"], norm_eps)
     u = gelu(_affine(h2, w["w_fc1"], w.get("b_fc1")))
-    y[rows] = xr + np.asarray(w["ls2"], np.float64) * _affine(u, w["w_fc2"], w.get("b_fc2"))
+    yr = xr + np.asarray(w["ls2"], np.float64) * _affine(u, w["w_fc2"], w.get("b_fc2"))
+    if subset:
+        return yr
+    y = x.copy()
+    y[rows] = yr
     return y
 
 

@@ -149,3 +149,24 @@ def test_camera_trunk_four_blocks():
     want = O.camera_trunk_forward(shape, feats, blocks, EPS)
     x0 = O.bf16_to_f64(feats)[O.register_tokens(shape)]
     _check(got, want, x0, np.arange(len(want)), scale=2.0)
+
+
+@pytest.mark.parametrize("mode,idx,count", [("frame", 2, 256), ("global", 2, 256), ("register", 4, 512)])
+def test_block_at_workload_size_sampled(mode, idx, count):
+    """Blocks at the benchmark sizes (24 x 1031 tokens for frame and global, the 500-frame workload for
+    register), compared with the oracle on sampled rows (every token still provides keys)."""
+    import torch
+    import vit_attention_b200 as V
+    shape = W.workload(idx).shape
+    w = W.make_transformer_block_weights(shape.H, 140 + idx)
+    x = W.make_tokens(shape, 150 + idx)
+    xd = _dev_bits(x)
+    ws = torch.empty(V.vggt_block_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+    V.vggt_block_forward(mode, shape, xd, _dev_weights(w), EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    pool = O.register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T)
+    rows = pool[W.query_subset(len(pool), count, 160 + idx)]
+    got = xd.view(shape.S * shape.T, -1)[torch.as_tensor(rows, device="cuda")].float().cpu().numpy().astype(np.float64)
+    want = O.block_forward(mode, shape, x, w, EPS, rows)
+    x0 = O.bf16_to_f64(x[rows])
+    _check(got, want, x0, np.arange(len(rows)))

@@ -134,3 +134,11 @@ def test_camera_trunk_reduces_to_register_blocks(wts, x):
     y = O.block_forward("register", SHAPE, y, w2, EPS)
     np.testing.assert_allclose(O.camera_trunk_forward(SHAPE, x, [wts, w2], EPS), y[sp], rtol=1e-12, atol=1e-12)
     assert O.CAMERA_TRUNK_BLOCKS == 4
+
+
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
+def test_row_subset_equals_rows_of_full_result(mode, wts, x):
+    full = O.block_forward(mode, SHAPE, x, wts, EPS)
+    pool = O.register_tokens(SHAPE) if mode == "register" else np.arange(SHAPE.S * SHAPE.T)
+    rows = pool[[0, 3, len(pool) - 1]]
+    np.testing.assert_allclose(O.block_forward(mode, SHAPE, x, wts, EPS, rows), full[rows], rtol=1e-12, atol=1e-12)
