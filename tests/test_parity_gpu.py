@@ -27,6 +27,9 @@ SMALL = [
     ("register", shp(40, 2, 17, 4, 4)),       # 680 special tokens: 6 tiles, ragged 40
     ("register", shp(3, 2, 5, 2, 3)),         # 15 special tokens: one small tile
     ("frame", shp(1, 1, 1, 1, 1)),            # T = 2
+    ("frame", shp(2, 2, 17, 64, 64)),         # T = 4113: high-resolution frames, 33 tiles x 65 key steps
+    ("register", shp(300, 2, 1, 2, 3)),       # camera token only: 300 special tokens
+    ("global", shp(1, 3, 17, 30, 40)),        # one frame of 1217 tokens, odd head count
 ]
 
 
