@@ -669,7 +669,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-queries", type=int, default=128, help="oracle sample size of the CPU baseline")
+    ap.add_argument("--cpu-queries", type=int, default=512, help="oracle sample size of the CPU baseline")
     ap.add_argument("--ref-queries", type=int, default=16, help="oracle queries per step of --impl reference")
     ap.add_argument("--workload", type=int, default=HEADLINE,
                     help="index of a global-mode workload (default: the S=100 headline; 2 = S=24 for profiling)")
