@@ -348,6 +348,18 @@ def run_ours(args):
                 "frac_of_burst_peak": core_tflops / peaks.get("bf16_tflops", peak),
                 "prologue_ms": pro_ms,
                 "prologue_hbm_gbs": (shape.S * shape.T * shape.H * 64 * 2 * 4) / (pro_ms / 1000) / 1e9}
+    # The softmax's exponentials are the kernel's other ceiling: one exp2 per score (N^2 H per call), 7/8 of
+    # them on the MUFU unit (16 results/clk/SM), 1/8 as a polynomial on the FMA pipe.
+    n_tok = shape.S * shape.T
+    exps = float(n_tok) * n_tok * shape.H
+    sm_mhz = (clk or {}).get("sm_mhz") or 0.0
+    n_sm = torch.cuda.get_device_properties(device).multi_processor_count
+    if sm_mhz > 0:
+        mufu_peak = 16.0 * n_sm * sm_mhz * 1e6
+        roofline["exp"] = {"achieved_per_s": exps / (core_ms / 1000.0), "mufu_share": 7 / 8,
+                           "mufu_peak_per_s": mufu_peak,
+                           "mufu_frac": exps * 7 / 8 / (core_ms / 1000.0) / mufu_peak,
+                           "clock_mhz": sm_mhz}
 
     # ---- e2e: scenes from pinned host buffers through vggt_attn_host_pipeline: every step's H2D of its
     # qkv and D2H of its output are inside the timed region, on copy streams that overlap the
