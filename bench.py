@@ -504,8 +504,15 @@ def sharded_timings(V, device, stream, qkv, prm, global_ms):
         t_pro = cuda_time_ms(pro, stream, 3)
         t_core = cuda_time_ms(core, stream, 3)
         assert V.vggt_attn_read_status(ws, stream) == 0
+        # fused form: the same keys read in place from `world` per-rank buffers (here all on this GPU)
+        ks = [k_send] * world
+        vs = [v_send] * world
+        fused = lambda: V.vggt_attn_global_shard_core_peers(local, world, ks, vs, out_r, ws, None, stream)  # noqa: E731
+        fused()
+        t_fused = cuda_time_ms(fused, stream, 3)
+        assert V.vggt_attn_read_status(ws, stream) == 0
         gather_bytes = 2 * (world - 1) * k_send.numel() * 2          # k and v blocks received per rank
-        res[f"world_{world}"] = {"rank_prologue_ms": t_pro, "rank_core_ms": t_core,
+        res[f"world_{world}"] = {"rank_prologue_ms": t_pro, "rank_core_ms": t_core, "rank_core_fused_ms": t_fused,
                                  "rank_compute_ms": t_pro + t_core,
                                  "speedup_vs_1gpu_global": global_ms / (t_pro + t_core),
                                  "allgather_bytes_per_rank": gather_bytes,

@@ -384,6 +384,22 @@ int vggt_attn_host_pipeline(int mode, const vggt_attn_shape* shape, int n_items,
  * every argument before enqueueing anything and allocate nothing;
  * vggt_attn_shard_buffers does no device work. */
 size_t vggt_attn_shard_workspace_size(const vggt_attn_shape* shape, int world);
+/* Fused form: no all-gather.  vggt_attn_global_shard_core_peers runs rank r's
+ * queries over the keys and values of every rank read where each rank's
+ * prologue left them: k_ranks[q] / v_ranks[q] (q = 0 .. world-1, world <= 8)
+ * are device addresses, valid in this process, of rank q's k_send / v_send
+ * (this rank's own, and the peers' mapped over NVLink, e.g. through CUDA IPC);
+ * each rank's block of keys starts a new 64-key step, so results agree with
+ * vggt_attn_global to rounding (bit for bit when world = 1).  The caller makes
+ * sure every rank's prologue has completed before any rank's core starts and
+ * that no prologue overwrites its buffers while a core may still read them.
+ * Its workspace needs only the status word, q plane and send buffers:
+ * vggt_attn_shard_fused_workspace_size(shape) bytes (the prologue accepts
+ * that size too). */
+size_t vggt_attn_shard_fused_workspace_size(const vggt_attn_shape* shape);
+int vggt_attn_global_shard_core_peers(const vggt_attn_shape* shape, int world, const void* const* k_ranks,
+                                      const void* const* v_ranks, void* out,
+                                      void* workspace, size_t workspace_bytes, void* cuda_stream);
 int vggt_attn_shard_buffers(const vggt_attn_shape* shape, int world, void* workspace, void** k_send,
                             void** v_send, void** k_all, void** v_all);
 int vggt_attn_global_shard_prologue(const vggt_attn_shape* shape, int world, const void* qkv,

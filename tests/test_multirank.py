@@ -37,7 +37,7 @@ def _worker(rank, world, port, results):
 def test_two_gloo_ranks_shard_and_reduce():
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_worker, args=(world, port, results), nprocs=world, join=True)
         res = dict(results)
@@ -84,7 +84,7 @@ def test_sharded_global_gathers_kv_in_rank_order():
     all ranks' key/value rows, rank r's block at token offset r * L."""
     world = 2
     port = _free_port()
-    with mp.Manager() as m:
+    with mp.get_context("spawn").Manager() as m:
         results = m.dict()
         mp.spawn(_gather_worker, args=(world, port, results), nprocs=world, join=True)
         res = dict(results)

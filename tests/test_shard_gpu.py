@@ -95,3 +95,103 @@ def test_single_rank_helper_without_process_group():
     ws = torch.empty(V.vggt_attn_shard_workspace_size(shape, 1), dtype=torch.uint8, device="cuda")
     global_attention_sharded(shape, dev["qkv"], dev["q_gamma"], dev["q_beta"], dev["k_gamma"], dev["k_beta"], out, ws)
     assert torch.equal(out.view(torch.int16), _run_global(shape, dev).view(torch.int16))
+
+
+# ------------------------------------------------------------------ fused form (keys read in place)
+def _fused_emulated(shape, dev, world):
+    """All ranks in this process: W prologues into W workspaces, then each rank's core reads the W send
+    buffers in place (on one GPU they are simply this GPU's memory)."""
+    import dataclasses
+    import torch
+    import vit_attention_b200 as V
+    local = dataclasses.replace(shape, S=shape.S // world)
+    wss, ks, vs = [], [], []
+    for r in range(world):
+        ws = torch.empty(V.vggt_attn_shard_fused_workspace_size(local), dtype=torch.uint8, device="cuda")
+        V.vggt_attn_global_shard_prologue(local, world, dev["qkv"][r * local.S:(r + 1) * local.S], dev["q_gamma"],
+                                          dev["q_beta"], dev["k_gamma"], dev["k_beta"], ws)
+        k_send, v_send, _, _ = V.vggt_attn_shard_buffers(local, world, ws)
+        wss.append(ws)
+        ks.append(k_send)
+        vs.append(v_send)
+    outs = []
+    for r in range(world):
+        out = torch.zeros((local.S, local.T, local.H, 64), dtype=torch.bfloat16, device="cuda")
+        V.vggt_attn_global_shard_core_peers(local, world, ks, vs, out, wss[r])
+        assert V.vggt_attn_read_status(wss[r]) == 0
+        outs.append(out)
+    return torch.cat(outs)
+
+
+FUSED = [(shp(6, 4, 5, 7, 9), 3), (shp(4, 2, 17, 10, 30), 2), (shp(8, 2, 5, 3, 4), 8)]
+
+
+@pytest.mark.parametrize("shape,world", FUSED, ids=[f"S{s.S}T{s.T}H{s.H}-w{w}" for s, w in FUSED])
+def test_fused_ranks_match_oracle(shape, world):
+    x = W.make_random_inputs(shape, 210 + shape.T)
+    dev = _dev(x)
+    got = _fused_emulated(shape, dev, world)
+    q = query_sample("global", shape, 1 << 62, 0)
+    assert_close(rows(got, shape, q), O.attn_global(shape, x, q), f"fused sharded global, {world} ranks")
+
+
+def test_fused_single_rank_equals_global_bitwise():
+    import torch
+    shape = shp(3, 4, 17, 10, 12)
+    x = W.make_random_inputs(shape, 220)
+    dev = _dev(x)
+    assert torch.equal(_fused_emulated(shape, dev, 1).view(torch.int16), _run_global(shape, dev).view(torch.int16))
+
+
+def _ipc_worker(rank, world, port, seed, results):
+    """One rank of a 2-process run on one GPU: the other rank's keys/values are read through a CUDA IPC
+    mapping of its workspace (no kernel waits on the other process; the ranks meet at host barriers)."""
+    import dataclasses
+    import datetime
+    import os
+    import sys
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    sys.path.insert(0, os.path.join(root, "tests"))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=120))
+    torch.cuda.set_device(0)
+    import vit_attention_b200 as V
+    import workloads as W
+    from parity import to_device
+    from vit_attention_b200.sharded import PeerShards
+    shape = W.Shape(S=4, T=68, H=4, n_special=5, grid_h=7, grid_w=9)
+    local = dataclasses.replace(shape, S=shape.S // world)
+    x = W.make_random_inputs(shape, seed)
+    qkv, prm = to_device(x)
+    ws = torch.empty(V.vggt_attn_shard_fused_workspace_size(local), dtype=torch.uint8, device="cuda")
+    peers = PeerShards(local, ws)
+    out = torch.zeros((local.S, local.T, local.H, 64), dtype=torch.bfloat16, device="cuda")
+    peers.attend(qkv[rank * local.S:(rank + 1) * local.S], prm["q_gamma"], prm["q_beta"], prm["k_gamma"],
+                 prm["k_beta"], out)
+    torch.cuda.synchronize()
+    results[rank] = (V.vggt_attn_read_status(ws), out.float().cpu().numpy())
+    dist.barrier()
+    del peers
+    dist.destroy_process_group()
+
+
+def test_fused_two_processes_share_one_gpu_through_ipc():
+    import socket
+    import numpy as np
+    import torch.multiprocessing as mp
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    seed = 230
+    with mp.get_context("spawn").Manager() as m:
+        results = m.dict()
+        mp.spawn(_ipc_worker, args=(2, port, seed, results), nprocs=2, join=True)
+        res = dict(results)
+    assert res[0][0] == 0 and res[1][0] == 0
+    shape = W.Shape(S=4, T=68, H=4, n_special=5, grid_h=7, grid_w=9)
+    x = W.make_random_inputs(shape, seed)
+    got = np.concatenate([res[0][1], res[1][1]]).reshape(-1, shape.H, 64).astype(np.float64)
+    assert_close(got, O.attn_global(shape, x), "fused sharded global over IPC, 2 processes")

@@ -91,6 +91,9 @@ _SIGNATURES = {
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     "vggt_attn_global_shard_prologue": (_int, [_shape_p, _int, _vp, _fp, _fp, _fp, _fp, _vp, _sz, _vp]),
     "vggt_attn_global_shard_core": (_int, [_shape_p, _int, _vp, _vp, _sz, _vp]),
+    "vggt_attn_shard_fused_workspace_size": (_sz, [_shape_p]),
+    "vggt_attn_global_shard_core_peers": (_int, [_shape_p, _int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp,
+                                                 _vp, _sz, _vp]),
     "vggt_camera_trunk_workspace_size": (_sz, [_shape_p]),
     "vggt_camera_trunk_forward": (_int, [_shape_p, _vp, _vp, ctypes.POINTER(vggt_block_weights), _int,
                                          ctypes.c_float, _vp, _sz, _vp]),
@@ -339,8 +342,29 @@ def vggt_attn_shard_buffers(shape, world: int, workspace):
     for p, rows in zip(ptrs, (n, n, world * n, world * n)):
         off = p.value - workspace.data_ptr()
         nbytes = rows * shape.H * 64 * 2
+        if off + nbytes > workspace.numel():     # a fused-size workspace has no gathered buffers
+            views.append(None)
+            continue
         views.append(workspace[off:off + nbytes].view(torch.bfloat16).view(rows, shape.H, 64))
     return tuple(views)
+
+
+def vggt_attn_shard_fused_workspace_size(shape) -> int:
+    return _lib.vggt_attn_shard_fused_workspace_size(ctypes.byref(make_shape(shape)))
+
+
+def vggt_attn_global_shard_core_peers(shape, world, k_ranks, v_ranks, out, workspace, workspace_bytes=None,
+                                      stream=None):
+    """Core of query-sharded global attention reading every rank's keys/values in place: k_ranks[r] /
+    v_ranks[r] are device addresses (ints or tensors) of rank r's send buffers, valid in this process."""
+    if len(k_ranks) != world or len(v_ranks) != world:
+        raise ValueError("one key and one value buffer per rank")
+    ks = (_vp * world)(*[_ptr(t) for t in k_ranks])
+    vs = (_vp * world)(*[_ptr(t) for t in v_ranks])
+    rc = _lib.vggt_attn_global_shard_core_peers(ctypes.byref(make_shape(shape)), world, ks, vs, _ptr(out),
+                                                _ptr(workspace), _nbytes(workspace, workspace_bytes),
+                                                _stream(stream))
+    _check(rc, "vggt_attn_global_shard_core_peers")
 
 
 def vggt_attn_global_shard_prologue(shape, world, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace,

@@ -90,6 +90,16 @@ struct CoreParams {
   int* status;
   unsigned long long timeout_ns;
   SgaParams sga;      // SGA configuration only
+  int rank_tokens;    // per-rank key blocks (RANKS configuration): keys per rank,
+  int rank_steps;     // and 64-key steps per rank (the last one ragged)
+};
+
+// Keys and values of a query-sharded global attention, one tensor map per
+// rank over that rank's own buffers ([L][H][64], this GPU's or a peer's).
+constexpr int kMaxRankMaps = 8;
+struct RankMaps {
+  CUtensorMap k[kMaxRankMaps];
+  CUtensorMap v[kMaxRankMaps];
 };
 
 namespace core {
@@ -114,13 +124,17 @@ constexpr uint32_t POLY_PAIR_MASK = 0x80u;
 // shape instead (attention_frame_persistent.cuh): its CTAs take tile after
 // tile and start the next tile's products during the last one's epilogue,
 // 2 % faster on the 500-frame workload.
-template <int NQ_, bool SGA_ = false, bool KTM_ = false>
+template <int NQ_, bool SGA_ = false, bool KTM_ = false, bool RANKS_ = false>
 struct CoreCfg {
   static constexpr int NQ = NQ_;
   static constexpr bool SGA = SGA_;   // subsampled global attention epilogue
   // Keys token-major, [Lk][H][64] like the values (query-sharded global mode:
   // the keys all ranks gathered), instead of one [B*Lk][64] plane per head.
   static constexpr bool KTM = KTM_;
+  // Keys in per-rank blocks read from each rank's buffers (RankMaps); every
+  // block starts a new 64-key step and its last step is masked to its length.
+  static constexpr bool RANKS = RANKS_;
+  static_assert(!RANKS_ || KTM_, "rank blocks are token-major");
   static constexpr int CTAS_PER_SM = NQ_ == 2 ? 1 : 2;
   static constexpr int STAGES = NQ_ == 2 ? 8 : 5;
   static constexpr int OFF_Q = 0;                                  // NQ tiles
@@ -366,6 +380,8 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     tc_fence_before();
     mbar_arrive(bar(BAR_Q_TMEM + tile));
   }
+  int jr = 0;   // step inside the current rank block (RANKS configuration)
+  (void)jr;
   for (int j = 0; j < n_kv; ++j) {
     const int buf = j & 1;
     const uint32_t s_addr = s_base + buf * BN;
@@ -381,7 +397,15 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     tmem_ld32(s_addr, sr[0]);
     tmem_ld32(s_addr + 32, sr[1]);
     tmem_wait_ld();
-    const int valid = p.Lk - j * BN;         // keys of this step that exist (>= BN except on the last)
+    // keys of this step that exist (>= BN except on the last step, or on each
+    // rank block's last step)
+    int valid;
+    if constexpr (C::RANKS) {
+      valid = p.rank_tokens - jr * BN;
+      if (++jr == p.rank_steps) jr = 0;
+    } else {
+      valid = p.Lk - j * BN;
+    }
     if (valid < BN) {                        // last step only (uniform branch)
 #pragma unroll
       for (int c = 0; c < 2; ++c)
@@ -492,10 +516,11 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
   }
 }
 
+// Body of the core kernels: k_maps / v_maps hold one tensor map (or, for the
+// RANKS configuration, one per rank).
 template <class C>
-__global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
-    attn_core_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                     const __grid_constant__ CUtensorMap tmap_v, const CoreParams p) {
+__device__ __forceinline__ void attn_core_body(const CUtensorMap* q_map, const CUtensorMap* k_maps,
+                                               const CUtensorMap* v_maps, const CoreParams& p) {
   using namespace core;
   VGGT_CORE_CFG_NAMES(C);
   extern __shared__ uint8_t smem_raw[];
@@ -530,9 +555,9 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
     }
     fence_mbar_init();
     *abort_flag = status_is_set(p.status) ? 1 : 0;  // another CTA already failed: skip the work
-    tma_prefetch_desc(&tmap_q);
-    tma_prefetch_desc(&tmap_k);
-    tma_prefetch_desc(&tmap_v);
+    tma_prefetch_desc(q_map);
+    tma_prefetch_desc(&k_maps[0]);
+    tma_prefetch_desc(&v_maps[0]);
   }
   for (int e = threadIdx.x; e < KV_BYTES / 16; e += blockDim.x)
     reinterpret_cast<uint4*>(smem + OFF_ONES)[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
@@ -567,8 +592,11 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
       for (int s = 0; s < STAGES; ++s) issued[s] = 0;
       mbar_arrive_expect_tx(bar(BAR_Q), n_tiles * Q_BYTES);
       for (int i = 0; i < n_tiles; ++i)
-        tma_load_3d(sbase + OFF_Q + i * Q_BYTES, &tmap_q, bar(BAR_Q), 0, q0 + i * BM, h * p.B + b);
+        tma_load_3d(sbase + OFF_Q + i * Q_BYTES, q_map, bar(BAR_Q), 0, q0 + i * BM, h * p.B + b);
       bool ok = true;
+      int kr = 0, jr = 0;   // rank block and step inside it (RANKS configuration)
+      (void)kr;
+      (void)jr;
       for (int j = 0; j < n_kv; ++j) {
         const int st = j % STAGES;
         if (j >= STAGES) {
@@ -577,11 +605,20 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
           if (!ok) break;
         }
         mbar_arrive_expect_tx(bar(BAR_KV_FULL + st), 2 * KV_BYTES);
-        if constexpr (C::KTM)
-          tma_load_4d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
-        else
-          tma_load_3d(sbase + OFF_K + st * KV_BYTES, &tmap_k, bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
-        tma_load_4d(sbase + OFF_V + st * KV_BYTES, &tmap_v, bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+        if constexpr (C::RANKS) {
+          tma_load_4d(sbase + OFF_K + st * KV_BYTES, &k_maps[kr], bar(BAR_KV_FULL + st), 0, h, jr * BN, 0);
+          tma_load_4d(sbase + OFF_V + st * KV_BYTES, &v_maps[kr], bar(BAR_KV_FULL + st), 0, h, jr * BN, 0);
+          if (++jr == p.rank_steps) {
+            jr = 0;
+            ++kr;
+          }
+        } else {
+          if constexpr (C::KTM)
+            tma_load_4d(sbase + OFF_K + st * KV_BYTES, &k_maps[0], bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+          else
+            tma_load_3d(sbase + OFF_K + st * KV_BYTES, &k_maps[0], bar(BAR_KV_FULL + st), 0, j * BN, h * p.B + b);
+          tma_load_4d(sbase + OFF_V + st * KV_BYTES, &v_maps[0], bar(BAR_KV_FULL + st), 0, h, j * BN, b);
+        }
         ++issued[st];
       }
       if (!ok) {
@@ -667,6 +704,22 @@ __global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
 }
 
 // Fault-path self-test: one bounded wait on a barrier nobody arrives at.
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
+    attn_core_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, const CoreParams p) {
+  attn_core_body<C>(&tmap_q, &tmap_k, &tmap_v, p);
+}
+
+// Query-sharded global attention with the keys and values of every rank read
+// in place (RANKS configuration; at most kMaxRankMaps ranks).
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, C::CTAS_PER_SM)
+    attn_core_ranks_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ RankMaps maps,
+                           const CoreParams p) {
+  attn_core_body<C>(&tmap_q, maps.k, maps.v, p);
+}
+
 __global__ void selftest_timeout_kernel(int* status, unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar_storage;
   __shared__ int abort_storage;

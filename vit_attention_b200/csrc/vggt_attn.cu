@@ -1200,10 +1200,14 @@ int check_shard_shape(const vggt_attn_shape* s, int world) {
   return check_shape(&whole, VGGT_ATTN_GLOBAL);   // token counts of the whole scene
 }
 
-int check_shard_ws(const vggt_attn_shape* s, int world, void* ws, size_t ws_bytes) {
+// fused_prefix: only the status word, q plane and send buffers are needed (the
+// prologue, and the core that reads every rank's send buffers in place).
+int check_shard_ws(const vggt_attn_shape* s, int world, void* ws, size_t ws_bytes, bool fused_prefix = false) {
   if (!ws) return VGGT_ATTN_ERR_INVALID_ARG;
   if (!aligned(ws, 256)) return VGGT_ATTN_ERR_MISALIGNED;
-  if (ws_bytes < shard_layout(s, world, nullptr).bytes) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  const ShardLayout L = shard_layout(s, world, nullptr);
+  const size_t need = fused_prefix ? static_cast<size_t>(reinterpret_cast<uintptr_t>(L.k_all)) : L.bytes;
+  if (ws_bytes < need) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
   return VGGT_ATTN_OK;
 }
 
@@ -1234,7 +1238,7 @@ extern "C" int vggt_attn_global_shard_prologue(const vggt_attn_shape* shape, int
                                                void* cuda_stream) {
   int rc = check_shard_shape(shape, world);
   if (rc) return rc;
-  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes))) return rc;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes, true))) return rc;
   if (!qkv || !q_gamma || !q_beta || !k_gamma || !k_beta) return VGGT_ATTN_ERR_INVALID_ARG;
   if (!aligned(qkv, 16) || !aligned(q_gamma, 16) || !aligned(q_beta, 16) || !aligned(k_gamma, 16) ||
       !aligned(k_beta, 16))
@@ -1388,4 +1392,77 @@ extern "C" int vggt_attn_host_pipeline(int mode, const vggt_attn_shape* shape, i
     for (int b = 0; b < 2; ++b)
       if (ev[k][b]) cudaEventDestroy(ev[k][b]);   // released once the recorded work completes
   return rc;
+}
+
+// ---------------------------------------------------------------------------
+// Query-sharded global attention, fused form: the core reads every rank's
+// keys and values where the ranks' prologues wrote them (peer memory over
+// NVLink for the other ranks), no gathered copy.
+extern "C" size_t vggt_attn_shard_fused_workspace_size(const vggt_attn_shape* shape) {
+  if (check_shard_shape(shape, 1) != VGGT_ATTN_OK) return 0;
+  return static_cast<size_t>(reinterpret_cast<uintptr_t>(shard_layout(shape, 1, nullptr).k_all));
+}
+
+extern "C" int vggt_attn_global_shard_core_peers(const vggt_attn_shape* shape, int world, const void* const* k_ranks,
+                                                 const void* const* v_ranks, void* out, void* workspace,
+                                                 size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if (world > vggt::kMaxRankMaps) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes, true))) return rc;
+  if (!out || !k_ranks || !v_ranks) return VGGT_ATTN_ERR_INVALID_ARG;
+  for (int r = 0; r < world; ++r) {
+    if (!k_ranks[r] || !v_ranks[r]) return VGGT_ATTN_ERR_INVALID_ARG;
+    if (!aligned(k_ranks[r], 16) || !aligned(v_ranks[r], 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  }
+  if (!aligned(out, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t out_bytes = static_cast<size_t>(shape->S) * shape->T * shape->H * 128;
+  if (overlaps(out, out_bytes, workspace, workspace_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  using C = vggt::CoreCfg<2, false, true, true>;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  const long long H = shape->H;
+  CUtensorMap mq;
+  {
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(L.L), static_cast<cuuint64_t>(H)};
+    const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(L.L) * 128};
+    const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};
+    if (!make_map(&mq, L.w.q, 3, dims, strides, box_q)) return VGGT_ATTN_ERR_CUDA;
+  }
+  vggt::RankMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  {
+    // rank r's keys and values, [L][H][64]: (dim, head, token, 1); rows past L read as zeros
+    const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L.L), 1};
+    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(L.L) * H * 128};
+    const cuuint32_t box[4] = {64, 1, vggt::core::BN, 1};
+    for (int r = 0; r < world; ++r)
+      if (!make_map(&maps.k[r], k_ranks[r], 4, dims, strides, box) ||
+          !make_map(&maps.v[r], v_ranks[r], 4, dims, strides, box))
+        return VGGT_ATTN_ERR_CUDA;
+  }
+  const int spr = static_cast<int>((L.L + vggt::core::BN - 1) / vggt::core::BN);
+  vggt::CoreParams p{};
+  p.L = static_cast<int>(L.L);
+  p.Lk = world * spr * vggt::core::BN;   // n_kv = world * spr steps
+  p.H = shape->H;
+  p.B = 1;
+  p.out_T = shape->T;
+  p.out_group = static_cast<int>(L.L);
+  p.out = static_cast<uint16_t*>(out);
+  p.status = L.w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  p.rank_tokens = static_cast<int>(L.L);
+  p.rank_steps = spr;
+  if (cudaFuncSetAttribute(vggt::attn_core_ranks_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_ALLOC) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  cudaFuncAttributes fa;   // the register split assumes the compiled count (see launch_core_cfg)
+  if (cudaFuncGetAttributes(&fa, vggt::attn_core_ranks_kernel<C>) != cudaSuccess || fa.numRegs < C::REGS_AT_LAUNCH)
+    return VGGT_ATTN_ERR_CUDA;
+  const long long n_q = (L.L + 2 * vggt::core::BM - 1) / (2 * vggt::core::BM);
+  const dim3 grid(static_cast<unsigned>(n_q), static_cast<unsigned>(H), 1);
+  vggt::attn_core_ranks_kernel<C><<<grid, C::THREADS, C::SMEM_ALLOC, static_cast<cudaStream_t>(cuda_stream)>>>(
+      mq, maps, p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }

@@ -8,6 +8,15 @@ attention core after it are the library's kernels (vggt_attn_global_shard_*).
 The collective is the only data-path communication: head-sharded global
 attention (each rank a subset of heads over all tokens) needs none and is plain
 vggt_attn_global on a head slice of qkv.
+
+Fused form (`PeerShards`): no gathered copy at all.  Every rank maps the
+others' workspaces once (CUDA IPC handles exchanged over the process group);
+after the prologues, one attention kernel per rank reads each rank's keys and
+values straight from that rank's send buffers -- peer loads over NVLink,
+tile by tile, overlapping the products (vggt_attn_global_shard_core_peers).
+The ranks meet at a host barrier after their prologues (the buffers are
+written) and after the core (they have been read) -- no kernel waits on
+another rank.
 """
 from __future__ import annotations
 
@@ -42,3 +51,50 @@ def global_attention_sharded(shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, 
         with torch.cuda.stream(s):
             gather_kv(k_send, v_send, k_all, v_all, group)
     V.vggt_attn_global_shard_core(shape, world, out, workspace, stream=stream)
+
+
+class PeerShards:
+    """This rank's view of every rank's send buffers for the fused form.
+
+    Built once per (workspace, shape): the workspace tensors of all ranks are
+    shared through CUDA IPC (torch's tensor reduction), so every rank holds a
+    mapping of every other rank's workspace.  ``group`` must be a CPU-capable
+    process group (gloo) or any group supporting ``all_gather_object``.
+    """
+
+    def __init__(self, shape, workspace, group=None):
+        import torch.distributed as dist
+        from torch.multiprocessing.reductions import reduce_tensor
+        import vit_attention_b200 as V
+        self.world = dist.get_world_size(group) if dist.is_initialized() else 1
+        self.rank = dist.get_rank(group) if dist.is_initialized() else 0
+        self.group = group
+        self.shape = shape
+        self.workspace = workspace
+        k_send, v_send, _, _ = V.vggt_attn_shard_buffers(shape, self.world, workspace)
+        k_off = k_send.data_ptr() - workspace.data_ptr()
+        v_off = v_send.data_ptr() - workspace.data_ptr()
+        if self.world == 1:
+            self.peers = [workspace]
+        else:
+            handles = [None] * self.world
+            dist.all_gather_object(handles, reduce_tensor(workspace), group=group)
+            self.peers = [workspace if r == self.rank else fn(*args) for r, (fn, args) in enumerate(handles)]
+        self.k_ptrs = [t.data_ptr() + k_off for t in self.peers]
+        self.v_ptrs = [t.data_ptr() + v_off for t in self.peers]
+
+    def attend(self, qkv, q_gamma, q_beta, k_gamma, k_beta, out, stream=None) -> None:
+        """This rank's rows of global attention over the whole scene (see global_attention_sharded)."""
+        import torch
+        import torch.distributed as dist
+        import vit_attention_b200 as V
+        V.vggt_attn_global_shard_prologue(self.shape, self.world, qkv, q_gamma, q_beta, k_gamma, k_beta,
+                                          self.workspace, stream=stream)
+        if self.world > 1:
+            (stream or torch.cuda.current_stream()).synchronize()
+            dist.barrier(group=self.group)            # every rank's keys and values are written
+        V.vggt_attn_global_shard_core_peers(self.shape, self.world, self.k_ptrs, self.v_ptrs, out, self.workspace,
+                                            stream=stream)
+        if self.world > 1:
+            (stream or torch.cuda.current_stream()).synchronize()
+            dist.barrier(group=self.group)            # and read: the next prologue may overwrite them
