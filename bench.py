@@ -476,6 +476,14 @@ def sga_timings(V, device, stream, qkv, prm, out, global_ms):
         nk = shape.S * (shape.n_special + ((shape.grid_h + s_ - 1) // s_) * ((shape.grid_w + s_ - 1) // s_))
         res[f"grid_{s_}x{s_}"] = {"ms": t, "kept_keys": nk, "speedup_vs_global": global_ms / t,
                                  "tflops_over_kept_keys": 4.0 * n * nk * 64 * shape.H / (t / 1000) / 1e12}
+        # descriptor attention over the same number of keys (window means instead of window corners)
+        fd = lambda: V.vggt_attn_global_desc(shape, s_, s_, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"],  # noqa: E731
+                                             prm["k_beta"], out, ws, None, stream)
+        fd()
+        td = cuda_time_ms(fd, stream, 5)
+        assert V.vggt_attn_read_status(ws, stream) == 0
+        res[f"desc_{s_}x{s_}"] = {"ms": td, "descriptors": nk, "speedup_vs_global": global_ms / td,
+                                 "tflops_over_descriptors": 4.0 * n * nk * 64 * shape.H / (td / 1000) / 1e12}
         del ws
     return res
 

@@ -255,6 +255,21 @@ int vggt_attn_block(int mode, const vggt_attn_shape* shape, const void* x,
  * vggt_attn_global_sga: arguments as vggt_attn_global plus s_h, s_w (1..1024);
  * writes all of `out`; asynchronous, validates before enqueueing. */
 size_t vggt_attn_sga_workspace_size(const vggt_attn_shape* shape, int s_h, int s_w);
+
+/* Descriptor attention (FlashVGGT article, abstract): each frame is
+ * compressed into descriptors -- its camera/register tokens, unchanged, and
+ * one descriptor per s_h x s_w window of its patch grid (windows tile the grid
+ * from (0, 0), the last ones may be smaller) whose key is the mean of the
+ * window's normalised, rotated keys and whose value is the mean of its
+ * values -- and every query (all S*T tokens, normalised and rotated as in
+ * global mode) attends to the descriptors of all frames.  s_h = s_w = 1 is
+ * global attention.  Arguments and workspace as vggt_attn_global_sga (the
+ * workspace size is vggt_attn_sga_workspace_size(shape, s_h, s_w)); writes
+ * all of `out`; asynchronous, validates before enqueueing. */
+int vggt_attn_global_desc(const vggt_attn_shape* shape, int s_h, int s_w, const void* qkv,
+                          const float* q_gamma, const float* q_beta,
+                          const float* k_gamma, const float* k_beta, void* out,
+                          void* workspace, size_t workspace_bytes, void* cuda_stream);
 int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s_w, const void* qkv,
                          const float* q_gamma, const float* q_beta,
                          const float* k_gamma, const float* k_beta, void* out,

@@ -99,6 +99,7 @@ _SIGNATURES = {
                                          ctypes.c_float, _vp, _sz, _vp]),
     "vggt_attn_sga_workspace_size": (_sz, [_shape_p, _int, _int]),
     "vggt_attn_global_sga": (_int, [_shape_p, _int, _int, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
+    "vggt_attn_global_desc": (_int, [_shape_p, _int, _int, _vp, _fp, _fp, _fp, _fp, _vp, _vp, _sz, _vp]),
 }
 for _name, (_res, _args) in _SIGNATURES.items():
     _f = getattr(_lib, _name)
@@ -404,3 +405,12 @@ def vggt_attn_host_pipeline(mode, shape, h_qkv, q_gamma, q_beta, k_gamma, k_beta
                                       sc if h2d_stream is None else _stream(h2d_stream),
                                       sc if d2h_stream is None else _stream(d2h_stream))
     _check(rc, "vggt_attn_host_pipeline")
+
+
+def vggt_attn_global_desc(shape, s_h, s_w, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace,
+                          workspace_bytes=None, stream=None):
+    """Descriptor attention: every query over the per-frame descriptors (special tokens, s_h x s_w window means)."""
+    rc = _lib.vggt_attn_global_desc(ctypes.byref(make_shape(shape)), s_h, s_w, _ptr(qkv), _ptr(q_gamma),
+                                    _ptr(q_beta), _ptr(k_gamma), _ptr(k_beta), _ptr(out), _ptr(workspace),
+                                    _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_global_desc")

@@ -16,6 +16,7 @@ namespace vggt {
 
 struct SgaGeometry {
   int N, Nk, H, T, n_special, grid_w, s_h, s_w, nw, kept_per_frame;
+  int grid_h;
 };
 
 // Flat token index (s*T + t) of the r-th kept key: frame r / kept_per_frame;
@@ -72,6 +73,48 @@ __global__ void __launch_bounds__(256) sga_sum_kernel(SgaGeometry g, const uint1
   }
   atomicAdd(sums + hd, ak);
   atomicAdd(sums + g.H * 64 + hd, av);
+}
+
+// Descriptor attention (FlashVGGT article, abstract): descriptor r of a
+// frame is one of its camera/register tokens, copied, or one s_h x s_w window
+// of its patch grid (windows tile the grid from (0, 0), edge windows smaller)
+// whose key is the mean of the window's normalised rotated keys and whose
+// value is the mean of its values (fp32 sums, one bf16 rounding).  Keys go to
+// [H][Nk][64], values to [Nk][H][64]; a block per descriptor, a thread per
+// (head, pair of dims).
+__global__ void __launch_bounds__(256) desc_pool_kernel(SgaGeometry g, const uint16_t* k_plane, const uint16_t* qkv,
+                                                        uint16_t* ks_plane, uint16_t* vs) {
+  for (int r = blockIdx.x; r < g.Nk; r += gridDim.x) {
+    const int s = r / g.kept_per_frame, u = r - s * g.kept_per_frame;
+    int r0 = 0, r1 = 1, c0 = 0, c1 = 1, t0 = u;     // special token: a 1 x 1 "window" at t0
+    if (u >= g.n_special) {
+      const int k = u - g.n_special;
+      const int kr = k / g.nw, kc = k - kr * g.nw;
+      r0 = kr * g.s_h;
+      r1 = min(r0 + g.s_h, g.grid_h);
+      c0 = kc * g.s_w;
+      c1 = min(c0 + g.s_w, g.grid_w);
+      t0 = g.n_special;
+    }
+    const float inv = 1.0f / static_cast<float>((r1 - r0) * (c1 - c0));
+    for (int e = threadIdx.x; e < g.H * 32; e += blockDim.x) {
+      const int h = e >> 5, d2 = e & 31;           // dims 2 d2, 2 d2 + 1 of head h
+      float k0 = 0.f, k1 = 0.f, v0 = 0.f, v1 = 0.f;
+      for (int rr = r0; rr < r1; ++rr)
+        for (int cc = c0; cc < c1; ++cc) {
+          const int tok = s * g.T + t0 + (u >= g.n_special ? rr * g.grid_w + cc : 0);
+          const uint32_t kw = reinterpret_cast<const uint32_t*>(k_plane + (static_cast<size_t>(h) * g.N + tok) * 64)[d2];
+          const uint32_t vw =
+              reinterpret_cast<const uint32_t*>(qkv + ((static_cast<size_t>(tok) * 3 + 2) * g.H + h) * 64)[d2];
+          k0 += __uint_as_float(kw << 16);
+          k1 += __uint_as_float(kw & 0xFFFF0000u);
+          v0 += __uint_as_float(vw << 16);
+          v1 += __uint_as_float(vw & 0xFFFF0000u);
+        }
+      reinterpret_cast<uint32_t*>(ks_plane + (static_cast<size_t>(h) * g.Nk + r) * 64)[d2] = pack_bf16x2(k0 * inv, k1 * inv);
+      reinterpret_cast<uint32_t*>(vs + (static_cast<size_t>(r) * g.H + h) * 64)[d2] = pack_bf16x2(v0 * inv, v1 * inv);
+    }
+  }
 }
 
 }  // namespace vggt

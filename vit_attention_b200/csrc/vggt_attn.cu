@@ -771,6 +771,7 @@ bool sga_layout(const vggt_attn_shape* s, int s_h, int s_w, void* ws, SgaLayout*
   g.grid_w = s->grid_w > 0 ? s->grid_w : 1;
   g.s_h = s_h;
   g.s_w = s_w;
+  g.grid_h = s->grid_h;
   const int nh = s->grid_h > 0 ? (s->grid_h + s_h - 1) / s_h : 0;
   g.nw = s->grid_w > 0 ? (s->grid_w + s_w - 1) / s_w : 0;
   g.kept_per_frame = s->n_special + nh * g.nw;
@@ -871,6 +872,69 @@ extern "C" int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s
            g.T, g.n_special, g.grid_w, g.s_h, g.s_w};
   ModeGeometry mg{1, g.N, g.N, 2};
   return launch_core_cfg<vggt::CoreCfg<2, true>>(mg, g.H, mq, mk, mv, p, st);
+}
+
+// ---------------------------------------------------------------------------
+// Descriptor attention (FlashVGGT article, abstract): every query over the
+// per-frame descriptors (special tokens, window means of the patch grid).
+extern "C" int vggt_attn_global_desc(const vggt_attn_shape* shape, int s_h, int s_w, const void* qkv,
+                                     const float* q_gamma, const float* q_beta, const float* k_gamma,
+                                     const float* k_beta, void* out, void* workspace, size_t workspace_bytes,
+                                     void* cuda_stream) {
+  int rc = check_shape(shape, VGGT_ATTN_GLOBAL);
+  if (rc) return rc;
+  if (s_h < 1 || s_w < 1 || s_h > 1024 || s_w > 1024) return VGGT_ATTN_ERR_INVALID_ARG;
+  const size_t need = vggt_attn_sga_workspace_size(shape, s_h, s_w);   // same layout: descriptors in place of kept keys
+  if (need == 0) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (!workspace) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (workspace_bytes < need) return VGGT_ATTN_ERR_WORKSPACE_TOO_SMALL;
+  if ((rc = check_prologue_args(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace,
+                                workspace_bytes)))
+    return rc;
+  if ((rc = check_core_args(VGGT_ATTN_GLOBAL, shape, qkv, out, workspace, workspace_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  SgaLayout L;
+  sga_layout(shape, s_h, s_w, workspace, &L);
+  const vggt::SgaGeometry& g = L.g;
+  cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  // 1. QK-LayerNorm + RoPE of every token; 2. the descriptors (window means).
+  if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, L.w, st))) return rc;
+  {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
+      return VGGT_ATTN_ERR_CUDA;
+    vggt::desc_pool_kernel<<<static_cast<unsigned>(std::min(g.Nk, sms * 16)), 256, 0, st>>>(
+        g, L.w.k, static_cast<const uint16_t*>(qkv), L.ks, L.vs);
+    if (cudaGetLastError() != cudaSuccess) return VGGT_ATTN_ERR_CUDA;
+  }
+  // 3. Plain attention of every query over the descriptors.
+  CUtensorMap mq, mk, mv;
+  {
+    const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};
+    const cuuint32_t box_k[3] = {64, vggt::core::BN, 1};
+    const cuuint64_t dq[3] = {64, static_cast<cuuint64_t>(g.N), static_cast<cuuint64_t>(g.H)};
+    const cuuint64_t sq[2] = {128, static_cast<cuuint64_t>(g.N) * 128};
+    const cuuint64_t dk[3] = {64, static_cast<cuuint64_t>(g.Nk), static_cast<cuuint64_t>(g.H)};
+    const cuuint64_t sk[2] = {128, static_cast<cuuint64_t>(g.Nk) * 128};
+    if (!make_map(&mq, L.w.q, 3, dq, sq, box_q) || !make_map(&mk, L.ks, 3, dk, sk, box_k)) return VGGT_ATTN_ERR_CUDA;
+    const cuuint32_t box_v[4] = {64, 1, vggt::core::BN, 1};
+    const cuuint64_t dv[4] = {64, static_cast<cuuint64_t>(g.H), static_cast<cuuint64_t>(g.Nk), 1};
+    const cuuint64_t sv[3] = {128, static_cast<cuuint64_t>(g.H) * 128, static_cast<cuuint64_t>(g.Nk) * g.H * 128};
+    if (!make_map(&mv, L.vs, 4, dv, sv, box_v)) return VGGT_ATTN_ERR_CUDA;
+  }
+  vggt::CoreParams p{};
+  p.L = g.N;
+  p.Lk = g.Nk;
+  p.H = g.H;
+  p.B = 1;
+  p.out_T = shape->T;
+  p.out_group = g.N;
+  p.out = static_cast<uint16_t*>(out);
+  p.status = L.w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  ModeGeometry mg{1, g.N, g.N, 2};
+  return launch_core_cfg<vggt::CoreCfg<2>>(mg, g.H, mq, mk, mv, p, st);
 }
 
 // ---------------------------------------------------------------------------
