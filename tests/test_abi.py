@@ -99,3 +99,44 @@ def test_valid_call_without_gpu_fails_loudly(V):
     with pytest.raises(V.VggtAttnError):
         V.vggt_attn_global(W.workload(0).shape, 4096, 8192, 8448, 8704, 8960, 1 << 30, 1 << 32,
                            V.vggt_attn_workspace_size(W.workload(0).shape, "global"), stream=0)
+
+
+def test_block_and_pipeline_validation_without_device(V):
+    """Argument errors of the newer entry points are caught on the host, before any device work."""
+    s = W.Shape(S=2, T=68, H=4, n_special=5, grid_h=7, grid_w=9)
+    good = {f: (1 << 20) + 256 * i for i, f in enumerate(V.BLOCK_WEIGHT_FIELDS)}
+    wsb = V.vggt_block_workspace_size(s, "frame")
+    assert wsb > 0 and V.vggt_block_workspace_size(W.Shape(S=2, T=68, H=2, n_special=5, grid_h=7, grid_w=9),
+                                                    "frame") == 0          # C = 128: not a multiple of 256
+    lib = V.library()
+    shape = V.make_shape(s)
+    x = 1 << 34
+    ws = 1 << 36
+
+    def block(weights, eps=1e-6, nbytes=wsb, xx=x):
+        w = V.make_block_weights(weights)
+        return lib.vggt_block_forward(0, ctypes.byref(shape), xx, ctypes.byref(w), eps, ws, nbytes, None)
+
+    assert block(dict(good, ls1=None)) == V.ERR_INVALID_ARG
+    assert block(dict(good, w_fc1=(1 << 20) + 8)) == V.ERR_MISALIGNED
+    assert block(good, eps=0.0) == V.ERR_INVALID_ARG
+    assert block(good, nbytes=wsb - 1) == V.ERR_WORKSPACE_TOO_SMALL
+    assert block(good, xx=ws + 256) == V.ERR_INVALID_ARG                   # x inside the workspace
+    assert block(dict(good, w_qkv=x)) == V.ERR_INVALID_ARG                 # a weight overlapping x
+    # the schedule: a register layer index out of range
+    w = V.make_block_weights(good)
+    arr = (V.vggt_block_weights * 1)(w)
+    regs = (ctypes.c_int * 1)(3)
+    assert lib.vggt_aggregator_forward(ctypes.byref(shape), x, arr, arr, 1, regs, 1, 1e-6, ws,
+                                       V.vggt_aggregator_workspace_size(s), None) == V.ERR_INVALID_ARG
+    # host pipeline: missing host pointers; sharded core: too many ranks for the fused form
+    qs = (ctypes.c_void_p * 1)(None)
+    assert lib.vggt_attn_host_pipeline(1, ctypes.byref(shape), 1, qs, 256, 512, 768, 1024, qs, ws,
+                                       V.vggt_attn_host_pipeline_workspace_size(s, "global"), None, None,
+                                       None) == V.ERR_INVALID_ARG
+    ks = (ctypes.c_void_p * 9)(*([1 << 24] * 9))
+    assert lib.vggt_attn_global_shard_core_peers(ctypes.byref(shape), 9, ks, ks, x, ws, 1 << 30,
+                                                 None) == V.ERR_UNSUPPORTED_SHAPE
+    # descriptor attention: window sizes must be >= 1
+    assert lib.vggt_attn_global_desc(ctypes.byref(shape), 0, 2, 4096, 256, 512, 768, 1024, x, ws, 1 << 30,
+                                     None) == V.ERR_INVALID_ARG
