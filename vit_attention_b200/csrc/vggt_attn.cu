@@ -1,5 +1,17 @@
 // Host side of libvggt_attn.so: argument validation, workspace layout, TMA
 // tensor maps and the kernel launches behind the C ABI in vggt_attn.h.
+//
+// Sections, in order:
+//   shape checks, workspace views, tensor maps, prologue / core launches
+//   attention entry points (frame, global, register, prologue, core, status)
+//   allocation-free entry point (static scratch)
+//   projections: vggt_linear, vggt_attn_qkv_proj, vggt_attn_block
+//   subsampled global attention (SGA) and descriptor attention
+//   transformer blocks and the alternating layer schedule
+//   camera-head trunk
+//   query-sharded global attention (gathered form)
+//   host-memory pipeline
+//   query-sharded global attention (fused form: every rank's keys in place)
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
