@@ -347,6 +347,19 @@ int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_bl
                             const vggt_block_weights* inter_blocks, int n_layers, const int* register_layers,
                             int n_register, float norm_eps, void* workspace, size_t workspace_bytes,
                             void* cuda_stream);
+/* vggt_aggregator_forward_cached: the same schedule, and for each layer
+ * cache_layers[i] (host array, n_cache entries) the layer's features are kept
+ * in cache_out[i] (device, bf16 [S][T][2C]): channels [0, C) the output of its
+ * frame block, channels [C, 2C) the output of its inter-frame block
+ * (Aggregator explainer, section 4: the cached layers 4, 11, 17 and 23 feed the
+ * heads with the frame and inter-frame outputs concatenated; the camera trunk
+ * takes the last layer's).  cache_out buffers must not overlap x or the
+ * workspace. */
+int vggt_aggregator_forward_cached(const vggt_attn_shape* shape, void* x, const vggt_block_weights* frame_blocks,
+                                   const vggt_block_weights* inter_blocks, int n_layers,
+                                   const int* register_layers, int n_register, const int* cache_layers,
+                                   int n_cache, void* const* cache_out, float norm_eps, void* workspace,
+                                   size_t workspace_bytes, void* cuda_stream);
 
 /* ------------------------------------------------------------------------
  * Host-memory pipeline: n_items independent calls of one mode (frame, global

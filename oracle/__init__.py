@@ -53,6 +53,7 @@ from .projection import attention_block, linear, projected_qkv  # noqa: F401
 from .sga import attn_global_sga, sga_kept_tokens  # noqa: F401
 from .descriptor import attn_global_desc, descriptor_windows  # noqa: F401
 from .block import (  # noqa: F401
+    CACHED_LAYERS,
     CAMERA_TRUNK_BLOCKS,
     N_LAYERS,
     camera_trunk_forward,

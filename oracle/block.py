@@ -11,7 +11,9 @@ Source, cited by page title and section:
        Q/K normalisation together with LayerScale (initial value 1e-5).
   [P1] section 2: the patch tokens come from a DINO-style ViT, whose block
        the Aggregator's blocks follow.
-  [P1] section 4: the camera head takes the first 17 tokens (camera +
+  [P1] section 4: only layers 4, 11, 17 and 23 are cached, each as the
+       frame-block and inter-frame-block outputs concatenated along channels
+       (2 x 1024); the camera head takes the first 17 tokens (camera +
        registers) of every frame from the last layer and mixes them across
        frames again with 4 self-attention blocks.
 
@@ -104,14 +106,27 @@ def block_forward(mode: str, shape, x, w, norm_eps: float, rows=None) -> np.ndar
     return y
 
 
-def aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, norm_eps: float) -> np.ndarray:
+CACHED_LAYERS = (4, 11, 17, 23)          # [P1] section 4
+
+
+def aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, norm_eps: float,
+                       cache_layers=()) -> np.ndarray:
     """Layer l: the frame block frame_blocks[l], then the inter-frame block
-    inter_blocks[l], in register mode if l is in register_layers, else global."""
+    inter_blocks[l], in register mode if l is in register_layers, else global.
+
+    With ``cache_layers``, returns ``(y, cache)`` where cache[l] is ``[S*T, 2C]``:
+    the layer's frame-block output and inter-frame-block output side by side
+    ([P1] section 4: the heads read the cached layers' concatenated outputs).
+    """
     y = bf16_to_f64(x) if x.dtype == np.uint16 else np.asarray(x, np.float64)
+    cache = {}
     for l, (fw, iw) in enumerate(zip(frame_blocks, inter_blocks)):
         y = block_forward("frame", shape, y, fw, norm_eps)
+        frame_out = y
         y = block_forward("register" if l in register_layers else "global", shape, y, iw, norm_eps)
-    return y
+        if l in cache_layers:
+            cache[l] = np.concatenate([frame_out, y], axis=1)
+    return (y, cache) if cache_layers else y
 
 
 CAMERA_TRUNK_BLOCKS = 4                  # [P1] section 4

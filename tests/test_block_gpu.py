@@ -170,3 +170,28 @@ def test_block_at_workload_size_sampled(mode, idx, count):
     want = O.block_forward(mode, shape, x, w, EPS, rows)
     x0 = O.bf16_to_f64(x[rows])
     _check(got, want, x0, np.arange(len(rows)))
+
+
+def test_aggregator_caches_layers_for_the_heads():
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(4, 4, 5, 4, 5)     # C = 256
+    fw = [W.make_transformer_block_weights(shape.H, 170 + l) for l in range(3)]
+    iw = [W.make_transformer_block_weights(shape.H, 180 + l) for l in range(3)]
+    x = W.make_tokens(shape, 190)
+    xd = _dev_bits(x).clone()
+    M, C = shape.S * shape.T, shape.H * 64
+    cache = {l: torch.full((M, 2 * C), -9.0, dtype=torch.bfloat16, device="cuda") for l in (0, 2)}
+    ws = torch.empty(V.vggt_aggregator_workspace_size(shape), dtype=torch.uint8, device="cuda")
+    V.vggt_aggregator_forward_cached(shape, xd, [_dev_weights(w) for w in fw], [_dev_weights(w) for w in iw], [1],
+                                     cache, EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    y, want = O.aggregator_forward(shape, x, fw, iw, [1], EPS, cache_layers=(0, 2))
+    # the last layer's inter-frame output is x itself
+    assert torch.equal(cache[2][:, C:].view(torch.int16), xd.view(torch.int16))
+    x0 = O.bf16_to_f64(x)
+    for l in (0, 2):
+        got = cache[l].float().cpu().numpy().astype(np.float64)
+        for half in (0, 1):
+            sl = slice(half * C, (half + 1) * C)
+            _check(got[:, sl], want[l][:, sl], x0, np.arange(M), scale=3.0)

@@ -142,3 +142,15 @@ def test_row_subset_equals_rows_of_full_result(mode, wts, x):
     pool = O.register_tokens(SHAPE) if mode == "register" else np.arange(SHAPE.S * SHAPE.T)
     rows = pool[[0, 3, len(pool) - 1]]
     np.testing.assert_allclose(O.block_forward(mode, SHAPE, x, wts, EPS, rows), full[rows], rtol=1e-12, atol=1e-12)
+
+
+def test_cached_layers_concatenate_frame_and_inter_outputs(wts, x):
+    w2 = W.make_transformer_block_weights(SHAPE.H, 46)
+    y, cache = O.aggregator_forward(SHAPE, x, [wts, w2], [w2, wts], [1], EPS, cache_layers=(0, 1))
+    f0 = O.block_forward("frame", SHAPE, x, wts, EPS)
+    g0 = O.block_forward("global", SHAPE, f0, w2, EPS)
+    f1 = O.block_forward("frame", SHAPE, g0, w2, EPS)
+    np.testing.assert_array_equal(cache[0], np.concatenate([f0, g0], axis=1))
+    np.testing.assert_array_equal(cache[1][:, :SHAPE.H * 64], f1)
+    np.testing.assert_array_equal(cache[1][:, SHAPE.H * 64:], y)
+    assert O.CACHED_LAYERS == (4, 11, 17, 23)

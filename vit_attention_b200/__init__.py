@@ -80,6 +80,10 @@ _SIGNATURES = {
     "vggt_block_forward": (_int, [_int, _shape_p, _vp, ctypes.POINTER(vggt_block_weights), ctypes.c_float, _vp, _sz,
                                   _vp]),
     "vggt_aggregator_workspace_size": (_sz, [_shape_p]),
+    "vggt_aggregator_forward_cached": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
+                                              ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int),
+                                              _int, ctypes.POINTER(ctypes.c_int), _int, ctypes.POINTER(_vp),
+                                              ctypes.c_float, _vp, _sz, _vp]),
     "vggt_aggregator_forward": (_int, [_shape_p, _vp, ctypes.POINTER(vggt_block_weights),
                                        ctypes.POINTER(vggt_block_weights), _int, ctypes.POINTER(ctypes.c_int), _int,
                                        ctypes.c_float, _vp, _sz, _vp]),
@@ -293,6 +297,25 @@ def vggt_block_forward(mode, shape, x, weights, norm_eps, workspace, workspace_b
 
 def vggt_aggregator_workspace_size(shape) -> int:
     return _lib.vggt_aggregator_workspace_size(ctypes.byref(make_shape(shape)))
+
+
+def vggt_aggregator_forward_cached(shape, x, frame_blocks, inter_blocks, register_layers, cache, norm_eps,
+                                   workspace, workspace_bytes=None, stream=None):
+    """vggt_aggregator_forward, also keeping the features of the layers in ``cache`` (a dict layer -> bf16
+    device tensor [S*T, 2C]): frame-block output in the first C channels, inter-frame-block output in the rest."""
+    n = len(frame_blocks)
+    if len(inter_blocks) != n:
+        raise ValueError("frame_blocks and inter_blocks must have one entry per layer")
+    fb = (vggt_block_weights * max(n, 1))(*[make_block_weights(w) for w in frame_blocks])
+    ib = (vggt_block_weights * max(n, 1))(*[make_block_weights(w) for w in inter_blocks])
+    regs = (ctypes.c_int * max(len(register_layers), 1))(*register_layers)
+    layers = sorted(cache)
+    cl = (ctypes.c_int * max(len(layers), 1))(*layers)
+    co = (_vp * max(len(layers), 1))(*[_ptr(cache[l]) for l in layers])
+    rc = _lib.vggt_aggregator_forward_cached(ctypes.byref(make_shape(shape)), _ptr(x), fb, ib, n, regs,
+                                             len(register_layers), cl, len(layers), co, norm_eps, _ptr(workspace),
+                                             _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_aggregator_forward_cached")
 
 
 def vggt_aggregator_forward(shape, x, frame_blocks, inter_blocks, register_layers, norm_eps, workspace,

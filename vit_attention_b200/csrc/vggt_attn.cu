@@ -1140,11 +1140,14 @@ extern "C" size_t vggt_aggregator_workspace_size(const vggt_attn_shape* shape) {
   return need;
 }
 
-extern "C" int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_block_weights* frame_blocks,
-                                       const vggt_block_weights* inter_blocks, int n_layers,
-                                       const int* register_layers, int n_register, float norm_eps, void* workspace,
-                                       size_t workspace_bytes, void* cuda_stream) {
+extern "C" int vggt_aggregator_forward_cached(const vggt_attn_shape* shape, void* x,
+                                              const vggt_block_weights* frame_blocks,
+                                              const vggt_block_weights* inter_blocks, int n_layers,
+                                              const int* register_layers, int n_register, const int* cache_layers,
+                                              int n_cache, void* const* cache_out, float norm_eps, void* workspace,
+                                              size_t workspace_bytes, void* cuda_stream) {
   if (n_layers < 0 || n_register < 0 || (n_register > 0 && !register_layers)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (n_cache < 0 || (n_cache > 0 && (!cache_layers || !cache_out))) return VGGT_ATTN_ERR_INVALID_ARG;
   if (n_layers > 0 && (!frame_blocks || !inter_blocks)) return VGGT_ATTN_ERR_INVALID_ARG;
   if (!std::isfinite(norm_eps) || !(norm_eps > 0.f)) return VGGT_ATTN_ERR_INVALID_ARG;
   int rc;
@@ -1161,17 +1164,44 @@ extern "C" int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, co
     if ((rc = check_block_weights(&frame_blocks[l], C, x, x_bytes, workspace, workspace_bytes)) ||
         (rc = check_block_weights(&inter_blocks[l], C, x, x_bytes, workspace, workspace_bytes)))
       return rc;
+  for (int i = 0; i < n_cache; ++i) {
+    if (cache_layers[i] < 0 || cache_layers[i] >= n_layers || !cache_out[i]) return VGGT_ATTN_ERR_INVALID_ARG;
+    if (!aligned(cache_out[i], 16)) return VGGT_ATTN_ERR_MISALIGNED;
+    if (overlaps(cache_out[i], 2 * x_bytes, x, x_bytes) || overlaps(cache_out[i], 2 * x_bytes, workspace, workspace_bytes))
+      return VGGT_ATTN_ERR_INVALID_ARG;
+  }
   if ((rc = check_device())) return rc;
   cudaStream_t st = static_cast<cudaStream_t>(cuda_stream);
+  const size_t row = static_cast<size_t>(C) * 2;
+  const size_t rows = static_cast<size_t>(shape->S) * shape->T;
+  // x into channels [half*C, (half+1)*C) of every cache buffer kept for layer l.
+  auto cache = [&](int l, int half) -> int {
+    for (int i = 0; i < n_cache; ++i)
+      if (cache_layers[i] == l &&
+          cudaMemcpy2DAsync(static_cast<uint8_t*>(cache_out[i]) + half * row, 2 * row, x, row, row, rows,
+                            cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+        return VGGT_ATTN_ERR_CUDA;
+    return VGGT_ATTN_OK;
+  };
   for (int l = 0; l < n_layers; ++l) {
     bool reg = false;
     for (int i = 0; i < n_register; ++i) reg = reg || register_layers[i] == l;
     if ((rc = run_block(VGGT_ATTN_FRAME, shape, x, &frame_blocks[l], norm_eps, workspace, l == 0, st))) return rc;
+    if ((rc = cache(l, 0))) return rc;
     if ((rc = run_block(reg ? VGGT_ATTN_REGISTER : VGGT_ATTN_GLOBAL, shape, x, &inter_blocks[l], norm_eps, workspace,
                         false, st)))
       return rc;
+    if ((rc = cache(l, 1))) return rc;
   }
   return VGGT_ATTN_OK;
+}
+
+extern "C" int vggt_aggregator_forward(const vggt_attn_shape* shape, void* x, const vggt_block_weights* frame_blocks,
+                                       const vggt_block_weights* inter_blocks, int n_layers,
+                                       const int* register_layers, int n_register, float norm_eps, void* workspace,
+                                       size_t workspace_bytes, void* cuda_stream) {
+  return vggt_aggregator_forward_cached(shape, x, frame_blocks, inter_blocks, n_layers, register_layers, n_register,
+                                        nullptr, 0, nullptr, norm_eps, workspace, workspace_bytes, cuda_stream);
 }
 
 // ---------------------------------------------------------------------------
