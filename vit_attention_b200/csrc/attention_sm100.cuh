@@ -1,8 +1,12 @@
 // Exact softmax attention core for head_dim 64 on sm_100a (tcgen05 + TMEM + TMA).
 //
 // One CTA computes NQ 128-query tiles of one (problem, head) (NQ = 2 in
-// global and register mode; NQ = 1 with two CTAs per SM in frame mode, see
-// CoreCfg; the text below describes NQ = 2):
+// global and register mode; frame mode runs the persistent one-tile kernel of
+// attention_frame_persistent.cuh with the same per-step code; the text below
+// describes NQ = 2).  Configurations (CoreCfg): SGA adds the subsampled global
+// attention terms in the epilogue, KTM reads keys token-major like values,
+// RANKS reads the keys and values of several ranks' buffers in turn
+// (attn_core_ranks_kernel, query-sharded global attention):
 //   O = softmax(Q K^T) V   over the problem's L keys.  Q arrives scaled by
 //   softmax_scale*log2(e) from the prologue, so scores are in base 2.
 // (VGGT-Omega Aggregator explainer, section 3: the frame / global / register
