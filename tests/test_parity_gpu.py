@@ -85,6 +85,30 @@ def test_frame_more_units_than_ctas(shape):
     check_mode("frame", shape, x)
 
 
+# ------------------------------------------------------------------ degenerate inputs
+def test_zero_variance_rows_and_uniform_attention():
+    """Rows whose q or k is constant over the head (zero variance: the LayerNorm output is beta, the
+    epsilon alone keeps it finite), and one head whose keys are all equal (every score of a query equal:
+    the output is the plain mean of v)."""
+    import numpy as np
+    shape = shp(2, 3, 5, 6, 7)
+    x = W.make_random_inputs(shape, 31)
+    qkv = x["qkv"]
+    qkv[0, :10, 0, 1] = W.f32_to_bf16_bits(np.full(64, 0.75, np.float32))     # constant q rows, head 1
+    qkv[1, 3:20, 1, 2] = W.f32_to_bf16_bits(np.full(64, -2.0, np.float32))    # constant k rows, head 2
+    qkv[:, :, 1, 0] = qkv[0, 0, 1, 0]                                          # head 0: one key for all tokens
+    x["k_gamma"][0] = 1.0
+    x["k_beta"][0] = 0.0
+    for mode in ("global", "frame", "register"):
+        check_mode(mode, shape, x)
+    # register mode has no RoPE: head 0's equal keys give every special query the mean of the special v
+    out = run_gpu("register", shape, x).float().cpu().numpy()
+    sp = O.register_tokens(shape)
+    got = out.reshape(-1, shape.H, 64)[sp, 0]
+    want = O.bf16_to_f64(qkv.reshape(-1, 3, shape.H, 64)[sp, 2, 0]).mean(axis=0)
+    assert np.abs(got - want[None]).max() <= 2e-2
+
+
 # ------------------------------------------------------------------ the workloads at full size (sampled)
 def test_workload1_frame_full():
     w = W.workload(1)
