@@ -56,23 +56,37 @@ __global__ void __launch_bounds__(256) sga_gather_kernel(SgaGeometry g, const ui
   }
 }
 
-// sums[0][h][d] += k over the discarded tokens, sums[1][h][d] += v; thread =
-// (h, d) = blockIdx.y * blockDim.x + threadIdx.x, blocks stride over tokens.
+// sums[0][h][d] += k over the discarded tokens, sums[1][h][d] += v.  A block
+// takes a contiguous range of tokens; thread e < 8H sums dims 8(e%8)..+7 of k
+// of head e/8 (one 16-byte load per token: the head rows of a token are whole
+// 128-byte lines), thread 8H + e the same dims of v; each thread adds its 8
+// partial sums into `sums` once at the end.
 __global__ void __launch_bounds__(256) sga_sum_kernel(SgaGeometry g, const uint16_t* k_plane, const uint16_t* qkv,
                                                       float* sums) {
-  const int hd = blockIdx.y * blockDim.x + threadIdx.x;
-  if (hd >= g.H * 64) return;
-  const int h = hd >> 6, d = hd & 63;
-  float ak = 0.f, av = 0.f;
-  for (int tok = blockIdx.x; tok < g.N; tok += gridDim.x) {
-    if (sga_is_kept(g, tok)) continue;   // uniform over the block
-    const uint16_t kb = k_plane[(static_cast<size_t>(h) * g.N + tok) * 64 + d];
-    const uint16_t vb = qkv[((static_cast<size_t>(tok) * 3 + 2) * g.H + h) * 64 + d];
-    ak += __uint_as_float(static_cast<uint32_t>(kb) << 16);
-    av += __uint_as_float(static_cast<uint32_t>(vb) << 16);
+  const int lanes = g.H * 8;                        // 16-byte chunks per token, for k and for v each
+  const int per_block = (g.N + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * per_block;
+  const int t1 = min(g.N, t0 + per_block);
+  for (int e = threadIdx.x; e < 2 * lanes; e += blockDim.x) {
+    const bool is_v = e >= lanes;
+    const int c = is_v ? e - lanes : e;             // chunk: head c / 8, dims 8 (c % 8) ..
+    const int h = c >> 3, d8 = c & 7;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int tok = t0; tok < t1; ++tok) {
+      if (sga_is_kept(g, tok)) continue;            // the same for every thread of the block
+      const uint4 w = is_v ? reinterpret_cast<const uint4*>(qkv + ((static_cast<size_t>(tok) * 3 + 2) * g.H + h) * 64)[d8]
+                           : reinterpret_cast<const uint4*>(k_plane + (static_cast<size_t>(h) * g.N + tok) * 64)[d8];
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        acc[2 * k] += __uint_as_float(ww[k] << 16);
+        acc[2 * k + 1] += __uint_as_float(ww[k] & 0xFFFF0000u);
+      }
+    }
+    float* dst = sums + (is_v ? g.H * 64 : 0) + h * 64 + d8 * 8;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) atomicAdd(dst + k, acc[k]);
   }
-  atomicAdd(sums + hd, ak);
-  atomicAdd(sums + g.H * 64 + hd, av);
 }
 
 // Descriptor attention (FlashVGGT article, abstract): descriptor r of a

@@ -846,9 +846,8 @@ extern "C" int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s
     if (cudaGetDevice(&dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1)
       return VGGT_ATTN_ERR_CUDA;
-    const unsigned ycount = static_cast<unsigned>((g.H * 64 + 255) / 256);
-    const unsigned xcount = static_cast<unsigned>(std::max(1, std::min(g.N, sms * 8 / static_cast<int>(ycount) + 1)));
-    vggt::sga_sum_kernel<<<dim3(xcount, ycount), 256, 0, st>>>(g, L.w.k, static_cast<const uint16_t*>(qkv), L.sums);
+    const unsigned blocks = static_cast<unsigned>(std::max(1, std::min(g.N, sms * 8)));   // contiguous token ranges
+    vggt::sga_sum_kernel<<<blocks, 256, 0, st>>>(g, L.w.k, static_cast<const uint16_t*>(qkv), L.sums);
     vggt::sga_gather_kernel<<<static_cast<unsigned>(std::min(g.Nk, sms * 16)), 256, 0, st>>>(
         g, L.w.k, static_cast<const uint16_t*>(qkv), L.ks, L.vs);
     if (cudaGetLastError() != cudaSuccess) return VGGT_ATTN_ERR_CUDA;

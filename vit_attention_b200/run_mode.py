@@ -23,6 +23,8 @@ def main(argv=None) -> int:
     ap.add_argument("--frames", type=int, default=0, help="override the frame count S (0: keep)")
     ap.add_argument("--calls", type=int, default=3, help="timed calls after one warm-up call")
     ap.add_argument("--block", action="store_true", help="run a whole transformer block instead of attention")
+    ap.add_argument("--sga", type=int, default=0, help="global mode as subsampled global attention, s x s grid")
+    ap.add_argument("--desc", type=int, default=0, help="global mode as descriptor attention, s x s windows")
     args = ap.parse_args(argv)
 
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
@@ -60,10 +62,18 @@ def main(argv=None) -> int:
         prm = [(1.0 if k % 2 == 0 else 0.0) + 0.1 * torch.randn((H, 64), generator=g, device="cuda")
                for k in range(4)]
         out = torch.empty((shape.S, shape.T, H, 64), dtype=torch.bfloat16, device="cuda")
-        ws = torch.empty(V.vggt_attn_workspace_size(shape, args.mode), dtype=torch.uint8, device="cuda")
+        if args.sga or args.desc:
+            sz = args.sga or args.desc
+            fn = V.vggt_attn_global_sga if args.sga else V.vggt_attn_global_desc
+            ws = torch.empty(V.vggt_attn_sga_workspace_size(shape, sz, sz), dtype=torch.uint8, device="cuda")
 
-        def call():
-            V.attend(args.mode, shape, qkv, *prm, out, ws)
+            def call():
+                fn(shape, sz, sz, qkv, *prm, out, ws)
+        else:
+            ws = torch.empty(V.vggt_attn_workspace_size(shape, args.mode), dtype=torch.uint8, device="cuda")
+
+            def call():
+                V.attend(args.mode, shape, qkv, *prm, out, ws)
 
     call()
     torch.cuda.synchronize()
@@ -74,7 +84,8 @@ def main(argv=None) -> int:
     t1.record()
     t1.synchronize()
     status = V.vggt_attn_read_status(ws)
-    print(json.dumps({"mode": args.mode, "block": args.block, "S": shape.S, "T": shape.T, "H": H,
+    print(json.dumps({"mode": args.mode, "block": args.block, "sga": args.sga, "desc": args.desc,
+                      "S": shape.S, "T": shape.T, "H": H,
                       "ms_per_call": t0.elapsed_time(t1) / max(args.calls, 1), "status": status}))
     return 0 if status == 0 else 1
 
