@@ -140,3 +140,18 @@ def test_block_and_pipeline_validation_without_device(V):
     # descriptor attention: window sizes must be >= 1
     assert lib.vggt_attn_global_desc(ctypes.byref(shape), 0, 2, 4096, 256, 512, 768, 1024, x, ws, 1 << 30,
                                      None) == V.ERR_INVALID_ARG
+
+
+def test_empty_and_oversized_shapes_are_rejected_on_the_host(V):
+    lib = V.library()
+    f = lib.vggt_attn_global
+    for S, T, ns, gh, gw in ((0, 69, 5, 8, 8), (2, 0, 0, 0, 0)):
+        s = W.Shape(S=S, T=T, H=4, n_special=ns, grid_h=gh, grid_w=gw)
+        assert V.vggt_attn_workspace_size(s, "global") == 0
+        assert _call(V, f, s, wsb=1 << 30) == V.ERR_UNSUPPORTED_SHAPE
+    # more tokens than the kernels' 32-bit token indices allow
+    huge = W.Shape(S=2_100_000, T=1031, H=16, n_special=17, grid_h=26, grid_w=39)
+    assert V.vggt_attn_workspace_size(huge, "global") == 0
+    assert _call(V, f, huge, wsb=1 << 40) == V.ERR_UNSUPPORTED_SHAPE
+    # zero heads
+    assert _call(V, f, W.Shape(S=2, T=69, H=0, n_special=5, grid_h=8, grid_w=8), wsb=1 << 30) == V.ERR_UNSUPPORTED_SHAPE
