@@ -317,3 +317,27 @@ def test_workloads_follow_page_facts():
         s = w.shape
         assert (s.grid_w, s.grid_h, s.n_special, s.T) == (gw, gh, ns, ns + gw * gh) == (39, 26, 17, 1031)
         assert s.H * s.head_dim == f["feature_dim"]["value"]
+
+
+# ------------------------------------------------------------------ property checks over random small shapes
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(S=st.integers(1, 3), H=st.integers(1, 2), ns=st.integers(1, 4), gh=st.integers(0, 4), gw=st.integers(1, 4),
+       seed=st.integers(0, 10_000))
+def test_mode_identities_on_random_shapes(S, H, ns, gh, gw, seed):
+    """For any small shape: each frame of frame mode is global attention over that frame alone, and
+    register mode equals global attention over the special tokens taken as their own sequence."""
+    import dataclasses
+    shape = W.Shape(S=S, T=ns + gh * gw, H=H, n_special=ns, grid_h=gh, grid_w=gw)
+    x = W.make_random_inputs(shape, seed)
+    fr = O.attn_frame(shape, x)
+    for s in range(S):
+        one = dataclasses.replace(shape, S=1)
+        xs = dict(x, qkv=x["qkv"][s:s + 1])
+        np.testing.assert_allclose(fr[s * shape.T:(s + 1) * shape.T], O.attn_global(one, xs), rtol=1e-12, atol=1e-12)
+    reg = O.attn_register(shape, x)
+    sp = dataclasses.replace(shape, T=ns, grid_h=0, grid_w=0)
+    xr = dict(x, qkv=np.ascontiguousarray(x["qkv"][:, :ns]))
+    np.testing.assert_allclose(reg, O.attn_global(sp, xr), rtol=1e-12, atol=1e-12)
