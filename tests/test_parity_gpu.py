@@ -139,3 +139,15 @@ def test_workload4_register_then_frame():
     out_f = run_gpu("frame", w.shape, dev_inputs=dev)
     q = query_sample("frame", w.shape, 4096, w.seed)
     assert_close(rows(out_f, w.shape, q), O.attn_frame(w.shape, x, q), "frame S=500")
+
+
+# ------------------------------------------------------------------ random small shapes
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=30, deadline=None)
+@given(mode=st.sampled_from(["frame", "global", "register"]), S=st.integers(1, 5), H=st.integers(1, 3),
+       ns=st.integers(1, 17), gh=st.integers(0, 12), gw=st.integers(1, 12), seed=st.integers(0, 10_000))
+def test_random_small_shapes_match_oracle(mode, S, H, ns, gh, gw, seed):
+    shape = shp(S, H, ns, gh, gw)
+    check_mode(mode, shape, W.make_random_inputs(shape, seed))
