@@ -195,3 +195,24 @@ def test_aggregator_caches_layers_for_the_heads():
         for half in (0, 1):
             sl = slice(half * C, (half + 1) * C)
             _check(got[:, sl], want[l][:, sl], x0, np.arange(M), scale=3.0)
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=8, deadline=None)
+@given(mode=st.sampled_from(["frame", "global", "register"]), S=st.integers(1, 4), H=st.sampled_from([4, 8]),
+       ns=st.integers(1, 8), gh=st.integers(0, 8), gw=st.integers(1, 8), seed=st.integers(0, 10_000))
+def test_random_block_shapes(mode, S, H, ns, gh, gw, seed):
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(S, H, ns, gh, gw)
+    w = W.make_transformer_block_weights(H, seed)
+    x = W.make_tokens(shape, seed + 1)
+    xd = _dev_bits(x).clone()
+    ws = torch.empty(V.vggt_block_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+    V.vggt_block_forward(mode, shape, xd, _dev_weights(w), EPS, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    got = xd.float().cpu().numpy().astype(np.float64)
+    rows_ = O.register_tokens(shape) if mode == "register" else np.arange(shape.S * shape.T)
+    _check(got, O.block_forward(mode, shape, x, w, EPS), O.bf16_to_f64(x), rows_)

@@ -54,3 +54,26 @@ def test_desc_workload2_sampled():
     got = _run(w.shape, to_device(x), 2, 2)
     q = query_sample("global", w.shape, 512, w.seed)
     assert_close(rows(got, w.shape, q), O.attn_global_desc(w.shape, x, 2, 2, q), "desc 2x2, 24 frames")
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=20, deadline=None)
+@given(S=st.integers(1, 4), H=st.integers(1, 2), ns=st.integers(1, 6), gh=st.integers(0, 9), gw=st.integers(1, 9),
+       s_h=st.integers(1, 4), s_w=st.integers(1, 4), seed=st.integers(0, 10_000))
+def test_random_shapes_and_windows(S, H, ns, gh, gw, s_h, s_w, seed):
+    """Descriptor and subsampled global attention on random shapes and window sizes (ragged edge windows)."""
+    import vit_attention_b200 as V
+    import torch
+    shape = shp(S, H, ns, gh, gw)
+    x = W.make_random_inputs(shape, seed)
+    dev = to_device(x)
+    q = query_sample("global", shape, 1 << 62, 0)
+    assert_close(rows(_run(shape, dev, s_h, s_w), shape, q), O.attn_global_desc(shape, x, s_h, s_w, q), "desc")
+    qkv, prm = dev
+    out = torch.zeros((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(V.vggt_attn_sga_workspace_size(shape, s_h, s_w), dtype=torch.uint8, device="cuda")
+    V.vggt_attn_global_sga(shape, s_h, s_w, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"], prm["k_beta"], out, ws)
+    assert V.vggt_attn_read_status(ws) == 0
+    assert_close(rows(out, shape, q), O.attn_global_sga(shape, x, s_h, s_w, q), "sga")
