@@ -195,3 +195,22 @@ def test_fused_two_processes_share_one_gpu_through_ipc():
     x = W.make_random_inputs(shape, seed)
     got = np.concatenate([res[0][1], res[1][1]]).reshape(-1, shape.H, 64).astype(np.float64)
     assert_close(got, O.attn_global(shape, x), "fused sharded global over IPC, 2 processes")
+
+
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=12, deadline=None)
+@given(world=st.integers(1, 8), frames_per_rank=st.integers(1, 3), H=st.integers(1, 2), ns=st.integers(1, 6),
+       gh=st.integers(0, 7), gw=st.integers(1, 7), seed=st.integers(0, 10_000))
+def test_random_sharded_shapes(world, frames_per_rank, H, ns, gh, gw, seed):
+    """Gathered and fused sharded forms over random rank counts and shapes (rank blocks of any length)."""
+    import torch
+    shape = shp(world * frames_per_rank, H, ns, gh, gw)
+    x = W.make_random_inputs(shape, seed)
+    dev = _dev(x)
+    want = _run_global(shape, dev)
+    assert torch.equal(_run_sharded(shape, dev, world).view(torch.int16), want.view(torch.int16))
+    got = _fused_emulated(shape, dev, world)
+    q = query_sample("global", shape, 1 << 62, 0)
+    assert_close(rows(got, shape, q), O.attn_global(shape, x, q), "fused sharded global")
