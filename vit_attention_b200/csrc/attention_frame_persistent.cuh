@@ -1,7 +1,7 @@
 // Frame-mode attention core with persistent CTAs (VGGT-Omega Aggregator
 // explainer, section 3, step 1: each frame's tokens attend within the frame).
 //
-// A frame problem has only ceil(T/64) = 17 key steps per 128-query tile, so a
+// A frame problem has only ceil(T/80) = 13 key steps per 128-query tile, so a
 // CTA that computes one tile spends a large share of its life starting up
 // (barrier set-up, TMEM allocation, first loads from HBM) and draining.  Here
 // each CTA (two per SM, 256 threads, 256 TMEM columns) walks the units
@@ -11,10 +11,15 @@
 // buffer and its K/V into the same ring, the softmax warps copy the next Q
 // into TMEM as soon as the current unit's last QK^T product has completed,
 // so the next unit's first products run during this unit's epilogue.  The
-// per-step work is that of attn_core_kernel (see attention_sm100.cuh): Q in
-// TMEM, two S buffers, PV with 16 ones columns for the row sums, online
-// softmax with a lazily moved reference max.  Barrier phases run on across
-// units.  Every wait is bounded.
+// per-step work is that of attn_core_kernel (see attention_sm100.cuh) -- Q in
+// TMEM, two S buffers, online softmax with a lazily moved reference max --
+// with two differences that fit the 256 TMEM columns of a CTA that shares its
+// SM: steps of 80 keys (2 x 80 S + 64 O + 32 Q columns; 9 MMAs per 80 keys
+// against 8 per 64, the per-instruction cost of these small products being
+// what paces the loop), and row sums kept in registers by the softmax threads
+// (fp32 sums of the probabilities before their rounding to bf16) instead of
+// 16 ones columns in the PV product.  Barrier phases run on across units.
+// Every wait is bounded.
 #pragma once
 
 #include <cstdint>
@@ -25,16 +30,17 @@ namespace vggt {
 
 namespace fp {
 using core::BM;
-using core::BN;
 using core::D;
-using core::KV_BYTES;
 using core::Q_BYTES;
+constexpr int BN = 80;                                  // keys per step
+constexpr int KV_BYTES = BN * D * 2;                    // 10 KB key or value tile
+constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
+constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);   // V is MN-major
 constexpr int STAGES = 4;
 constexpr int OFF_Q = 0;                                // two Q buffers
 constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
 constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
-constexpr int OFF_ONES = OFF_V + STAGES * KV_BYTES;
-constexpr int OFF_BAR = OFF_ONES + KV_BYTES;
+constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
 enum {
   BAR_Q_FULL = 0,                       // [Q buffer]
   BAR_Q_EMPTY = BAR_Q_FULL + 2,         // [Q buffer]
@@ -51,18 +57,35 @@ enum {
 };
 constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;          // tmem slot, abort flag
 constexpr int SMEM_BYTES = OFF_MISC + 16;
-constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+constexpr int SMEM_ALLOC = SMEM_BYTES;   // base declared 1024-aligned; checked at entry
 constexpr int THREADS = 256;
 constexpr int CTAS_PER_SM = 2;
 constexpr uint32_t TMEM_COLS = 256;
-constexpr uint32_t COL_O = 128;                         // S buffers at 0 and 64
-constexpr uint32_t COL_Q = COL_O + core::NV;
+constexpr uint32_t COL_O = 2 * BN;                      // S buffers at 0 and 80
+constexpr uint32_t COL_Q = COL_O + D;
 constexpr int REGS_AT_LAUNCH = 128;
 constexpr int REGS_PRODUCER = 56;
 constexpr int REGS_SOFTMAX = 200;
 static_assert(REGS_PRODUCER * 128 + REGS_SOFTMAX * 128 <= REGS_AT_LAUNCH * THREADS, "register split too large");
-static_assert(SMEM_ALLOC * CTAS_PER_SM <= 227 * 1024, "two CTAs per SM");
+// 228 KB of shared memory per SM, 1 KB of it reserved per resident CTA
+static_assert((SMEM_ALLOC + 1024) * CTAS_PER_SM <= 228 * 1024, "two CTAs per SM");
+static_assert(COL_Q + 32 <= TMEM_COLS, "TMEM layout");
 }  // namespace fp
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
 
 struct FrameUnits {
   int n_qt;       // 128-query tiles per (frame, head)
@@ -135,6 +158,7 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
     q_ready = false;
     const int kv0 = i * n_kv;
     float m_run = -INFINITY;
+    float l_run = 0.f;
     for (int j = 0; j < n_kv; ++j) {
       const int g = G + j;
       const int buf = g & 1;
@@ -145,23 +169,22 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
       // S(j) complete => PV(j-2) complete: its K/V stage is free.
       if (j >= 2 && leader) mbar_arrive(bar(BAR_KV_EMPTY + (kv0 + j - 2) % STAGES));
       tc_fence_after();
-      uint32_t sr[2][32];
-      tmem_ld32(s_addr, sr[0]);
-      tmem_ld32(s_addr + 32, sr[1]);
+      uint32_t sr[BN];
+      tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(sr));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
+      tmem_ld16(s_addr + 64, sr + 64);
       tmem_wait_ld();
       const int valid = p.Lk - j * BN;
       if (valid < BN) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e >= valid) sr[c][e] = __float_as_uint(-INFINITY);
+        for (int e = 0; e < BN; ++e)
+          if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
       }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < 32; e += 2) {
-        mx0 = max3f(mx0, __uint_as_float(sr[0][e]), __uint_as_float(sr[0][e + 1]));
-        mx1 = max3f(mx1, __uint_as_float(sr[1][e]), __uint_as_float(sr[1][e + 1]));
+      for (int e = 0; e < BN; e += 4) {
+        mx0 = max3f(mx0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+        mx1 = max3f(mx1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
       }
       const float tile_max = fmaxf(mx0, mx1);
       const bool move = (j == 0) || (tile_max > m_run + core::RESCALE_THRESHOLD);
@@ -171,23 +194,26 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
         m_run = tile_max;
       }
       const float neg_m = -m_run;
+      {
+        uint32_t pk[BN / 2];
+        float l0 = 0.f, l1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < BN; e += 2) {
           float x0, x1, p0, p1;
-          add_x2(__uint_as_float(sr[c][e]), __uint_as_float(sr[c][e + 1]), neg_m, neg_m, x0, x1);
-          const int pair = (c * 32 + e) >> 1;
+          add_x2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), neg_m, neg_m, x0, x1);
+          const int pair = e >> 1;
           if ((core::POLY_PAIR_MASK >> (pair & 7)) & 1u) {
             exp2_poly_x2(x0, x1, p0, p1, pc);
           } else {
             p0 = ex2_approx(x0);
             p1 = ex2_approx(x1);
           }
+          add_x2(l0, l1, p0, p1, l0, l1);
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tmem_st16(s_addr + c * 16, pk);
+        l_run = l_run * alpha + (l0 + l1);
+        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(pk));
+        tmem_st8(s_addr + 32, pk + 32);
       }
       // Rescale O after PV(j-1) (S(j+1) was issued after it; past the unit's
       // last S, the unit's first PV_DONE commit says so).
@@ -199,19 +225,16 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
-        uint32_t orr[2][32], osum;
+        uint32_t orr[2][32];
         tmem_ld32(o_addr, orr[0]);
         tmem_ld32(o_addr + 32, orr[1]);
-        tmem_ld1(o_addr + D, osum);
         tmem_wait_ld();
 #pragma unroll
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[c][e] = __float_as_uint(__uint_as_float(orr[c][e]) * alpha);
-        osum = __float_as_uint(__uint_as_float(osum) * alpha);
         tmem_st32(o_addr, orr[0]);
         tmem_st32(o_addr + 32, orr[1]);
-        tmem_st1(o_addr + D, osum);
       }
       tmem_wait_st();
       tc_fence_before();
@@ -231,16 +254,15 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
     tc_fence_after();
     if (leader)
       for (int j = n_kv > 2 ? n_kv - 2 : 0; j < n_kv; ++j) mbar_arrive(bar(BAR_KV_EMPTY + (kv0 + j) % STAGES));
-    uint32_t orr[2][32], osum;
+    uint32_t orr[2][32];
     tmem_ld32(o_addr, orr[0]);
     tmem_ld32(o_addr + 32, orr[1]);
-    tmem_ld1(o_addr + D, osum);
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(bar(BAR_O_FREE));
     const int qi = q0 + row;
     if (qi < p.L) {
-      const float inv = 1.f / __uint_as_float(osum);
+      const float inv = 1.f / l_run;
       const long long out_row = static_cast<long long>(b) * p.out_T +
                                 static_cast<long long>(qi / p.out_group) * p.out_T + (qi % p.out_group);
       uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D);
@@ -269,11 +291,13 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
                                  const __grid_constant__ CUtensorMap tmap_v, const CoreParams p,
                                  const FrameUnits fu) {
   using namespace fp;
-  using core::IDESC_PV;
-  using core::IDESC_QK;
   using core::NV;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = smem_raw;
+  if ((smem_addr(smem_raw) & 1023u) != 0) {   // the tiles need 1024-byte alignment and there is no slack
+    if (threadIdx.x == 0) record_error(p.status, VGGT_ATTN_ERR_CUDA, 0x6F0u);
+    return;
+  }
   const uint32_t sbase = smem_addr(smem);
   const uint32_t bar0 = sbase + OFF_BAR;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
@@ -307,9 +331,6 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
   }
-  for (int e = threadIdx.x; e < KV_BYTES / 16; e += blockDim.x)
-    reinterpret_cast<uint4*>(smem + OFF_ONES)[e] = make_uint4(0x3F803F80u, 0x3F803F80u, 0x3F803F80u, 0x3F803F80u);
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   if (warp == 1) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
     tmem_relinquish();
@@ -382,7 +403,7 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
       };
       auto issue_pv = [&](int g, int k, bool first) {   // O (+)= P(g) [V(k) | 1]
         const uint32_t v_addr = sbase + OFF_V + (k % STAGES) * KV_BYTES;
-        const uint64_t v = smem_desc_sw128(v_addr, sbase + OFF_ONES - v_addr, 1024);
+        const uint64_t v = smem_desc_sw128(v_addr, KV_BYTES, 1024);   // N = 64: one swizzle atom wide
         const uint32_t a = tmem + (g & 1) * BN;
 #pragma unroll
         for (int kk = 0; kk < BN / 16; ++kk)

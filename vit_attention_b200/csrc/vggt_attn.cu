@@ -264,16 +264,18 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
                 cudaStream_t stream) {
   const ModeGeometry g = geometry(s, mode);
   CUtensorMap mq, mk, mv;
+  // keys per step: 80 in the frame kernel, 64 in the others
+  const cuuint32_t kv_rows = mode == VGGT_ATTN_FRAME ? vggt::fp::BN : vggt::core::BN;
   {
     const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(g.L), static_cast<cuuint64_t>(g.B * s->H)};
     const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(g.L) * 128};
     const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};   // one query tile
-    const cuuint32_t box_k[3] = {64, vggt::core::BN, 1};   // one key tile
+    const cuuint32_t box_k[3] = {64, kv_rows, 1};          // one key tile
     if (!make_map(&mq, w.q, 3, dims, strides, box_q) || !make_map(&mk, w.k, 3, dims, strides, box_k))
       return VGGT_ATTN_ERR_CUDA;
   }
   {
-    const cuuint32_t box[4] = {64, 1, vggt::core::BN, 1};  // one value tile
+    const cuuint32_t box[4] = {64, 1, kv_rows, 1};         // one value tile
     if (mode == VGGT_ATTN_REGISTER) {  // gathered v: [L][H][64]
       const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(s->H), static_cast<cuuint64_t>(g.L), 1};
       const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(s->H) * 128,
