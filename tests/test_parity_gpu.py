@@ -30,6 +30,10 @@ SMALL = [
     ("frame", shp(2, 2, 17, 64, 64)),         # T = 4113: high-resolution frames, 33 tiles x 65 key steps
     ("register", shp(300, 2, 1, 2, 3)),       # camera token only: 300 special tokens
     ("global", shp(1, 3, 17, 30, 40)),        # one frame of 1217 tokens, odd head count
+    ("frame", shp(2, 2, 5, 5, 15)),           # T = 80: exactly one frame-kernel key step (80 keys)
+    ("frame", shp(2, 2, 1, 8, 10)),           # T = 81: one full step and a 1-key step
+    ("frame", shp(2, 2, 5, 5, 31)),           # T = 160: exactly two steps
+    ("frame", shp(2, 2, 1, 10, 16)),          # T = 161: two full steps and a 1-key step
 ]
 
 
