@@ -211,7 +211,10 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
           add_x2(l0, l1, p0, p1, l0, l1);
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
+        // Row sum: this step's fp32 probabilities (two add chains) on top of
+        // the running sum, which moves with the reference max as O does.
         l_run = l_run * alpha + (l0 + l1);
+        // P (80 keys -> 40 bf16-pair columns) overwrites the first 40 columns of this S buffer.
         tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(pk));
         tmem_st8(s_addr + 32, pk + 32);
       }
