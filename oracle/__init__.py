@@ -20,7 +20,7 @@ Aggregator explainer, sections 2 and 3):
      frame (one frame), global (all S*T tokens), register (the n_special
      camera + register tokens of every frame; section 3, modes 1 and 2).
 
-Readings where the pages are silent (each is listed in the design doc):
+Readings where the pages are silent:
   * LayerNorm uses the biased variance and an epsilon passed by the caller
     (1e-5 by default).
   * RoPE: dims [0, 32) use the patch row, dims [32, 64) the patch column;

@@ -17,7 +17,7 @@ Source, cited by page title and section:
        registers) of every frame from the last layer and mixes them across
        frames again with 4 self-attention blocks.
 
-Readings where the page is silent (listed in the design doc):
+Readings where the page is silent:
   * A block is the pre-norm transformer block of a DINO-style ViT:
         x <- x + ls1 * proj(attention(qkv(norm1(x))))
         x <- x + ls2 * fc2(GELU(fc1(norm2(x))))

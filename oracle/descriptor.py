@@ -7,7 +7,7 @@ Source, cited by page title and section:
        cross-attention between the full set of image tokens (queries) and the
        descriptors (keys and values).
 
-Readings where the page is silent (listed in the design doc):
+Readings where the page is silent:
   * a frame's descriptors are its camera/register tokens, unchanged, plus one
     descriptor per s_h x s_w window of the patch grid (windows tile the grid
     from (0, 0); the last row/column of windows may be smaller) whose key is

@@ -6,7 +6,7 @@ Source, cited by page title and section:
        q, k and v (one linear projection, then the per-head QK-norm and RoPE of
        the attention core) and maps the attention output back to C channels.
 
-Readings where the page is silent (listed in the design doc): the projections are
+Readings where the page is silent: the projections are
 nn.Linear maps y = x W^T + b with W stored [out_features][in_features]; the
 3C outputs of the QKV projection are ordered [q | k | v], each [H][64].
 """

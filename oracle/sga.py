@@ -7,7 +7,7 @@ Source, cited by page title and section:
        while every query is kept; each token keeps its diagonal self-attention;
        all discarded columns are stood in for by one mean key-value pair.
 
-Readings where the page is silent (listed in the design doc):
+Readings where the page is silent:
   * kept keys K = every camera/register token of every frame, plus the patch
     tokens at (row, col) with row % s_h == 0 and col % s_w == 0 (the first
     token of each window), in every frame;
