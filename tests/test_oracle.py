@@ -76,7 +76,7 @@ def test_layer_norm_matches_torch_fp64():
 
 
 # ---------------------------------------------------------------- 2D RoPE
-@pytest.mark.parametrize("idx", [0, 1, 2])
+@pytest.mark.parametrize("idx", [0, 1, 2, 3, 4])
 def test_rope_golden_unit_vectors(idx):
     case = json.load(open(os.path.join(GOLDEN, "worked_examples.json")))["rope"][idx]
     y = O.rope_2d(unit(case["x_unit_dim"]), case["row"], case["col"], case["base"])
@@ -90,6 +90,15 @@ def test_rope_frequencies_closed_form():
     om = O.rope_frequencies(100.0)
     np.testing.assert_allclose(om, [100.0 ** (-j / 16) for j in range(16)], rtol=1e-15)
     assert om[0] == 1.0 and abs(om[8] - 0.1) < 1e-16
+
+
+@pytest.mark.parametrize("base,j,want", [(16.0, 4, 0.5), (16.0, 8, 0.25), (16.0, 12, 0.125),
+                                         (10000.0, 8, 0.01), (10000.0, 4, 0.1), (10.0, 16 - 1, 10.0 ** (-15 / 16))])
+def test_rope_frequencies_other_bases(base, j, want):
+    # omega_j = base^(-2j/32): powers of two for base 16, powers of ten for base 10^4
+    om = O.rope_frequencies(base)
+    assert om[0] == 1.0
+    assert abs(om[j] - want) <= 1e-15 * want
 
 
 def test_rope_matches_complex_rotation():
@@ -186,6 +195,25 @@ def test_attention_mask_removes_keys():
                                O.softmax_attention(q, k[3:7], v[3:7], 0.3), rtol=1e-13)
 
 
+def test_explicit_softmax_scale_golden():
+    case = json.load(open(os.path.join(GOLDEN, "worked_examples.json")))["pipeline_scale"][0]
+    shape = W.Shape(**case["shape"])
+    assert O.resolved_scale(shape) == 0.05
+    assert O.resolved_scale(W.Shape(**{**case["shape"], "softmax_scale": 0.0})) == 0.125
+    a = np.array([1.0, -1.0] * 32, dtype=np.float32)
+    b = np.array([1.0, 1.0, -1.0, -1.0] * 16, dtype=np.float32)
+    f = np.zeros((1, 2, 3, 1, 64), dtype=np.float32)
+    f[0, 0, 0, 0] = f[0, 0, 1, 0] = a
+    f[0, 1, 0, 0] = f[0, 1, 1, 0] = b
+    f[0, 0, 2, 0] = 1.0
+    x = {"qkv": W.f32_to_bf16_bits(f), "q_gamma": np.ones((1, 64), np.float32), "q_beta": np.zeros((1, 64), np.float32),
+         "k_gamma": np.ones((1, 64), np.float32), "k_beta": np.zeros((1, 64), np.float32)}
+    env = {"exp": math.exp}
+    out = O.attn_global(shape, x)
+    np.testing.assert_allclose(out[0, 0], eval(case["expected_out0"], env), rtol=1e-14)
+    np.testing.assert_allclose(out[1, 0], eval(case["expected_out1"], env), rtol=1e-13)
+
+
 # ---------------------------------------------------------------- whole pipeline (tiny)
 def _torch_pipeline(shape, x, mode):
     """Independent restatement with torch ops + complex RoPE + SDPA (fp64)."""
@@ -205,14 +233,17 @@ def _torch_pipeline(shape, x, mode):
             for arr in (q, k):
                 z = torch.complex(arr[:, t, :, half:half + 16], arr[:, t, :, half + 16:half + 32]) * rot
                 arr[:, t, :, half:half + 16], arr[:, t, :, half + 16:half + 32] = z.real, z.imag
+    sdpa_kw = {"scale": shape.softmax_scale} if shape.softmax_scale > 0 else {}   # SDPA's default is 1/sqrt(64)
     if mode == "frame":
-        o = torch.nn.functional.scaled_dot_product_attention(*(a.permute(0, 2, 1, 3) for a in (q, k, v)))
+        o = torch.nn.functional.scaled_dot_product_attention(*(a.permute(0, 2, 1, 3) for a in (q, k, v)), **sdpa_kw)
         return o.permute(0, 2, 1, 3).reshape(S * T, H, 64).numpy()
     if mode == "global":
-        o = torch.nn.functional.scaled_dot_product_attention(*(a.reshape(S * T, H, 64).permute(1, 0, 2) for a in (q, k, v)))
+        o = torch.nn.functional.scaled_dot_product_attention(*(a.reshape(S * T, H, 64).permute(1, 0, 2) for a in (q, k, v)),
+                                                             **sdpa_kw)
         return o.permute(1, 0, 2).numpy()
     ns = shape.n_special
-    o = torch.nn.functional.scaled_dot_product_attention(*(a[:, :ns].reshape(S * ns, H, 64).permute(1, 0, 2) for a in (q, k, v)))
+    o = torch.nn.functional.scaled_dot_product_attention(*(a[:, :ns].reshape(S * ns, H, 64).permute(1, 0, 2) for a in (q, k, v)),
+                                                         **sdpa_kw)
     return o.permute(1, 0, 2).numpy()
 
 
@@ -220,6 +251,14 @@ def _torch_pipeline(shape, x, mode):
 def test_pipeline_matches_torch_restatement(mode):
     shape = tiny_shape(S=3, H=2)
     x = W.make_random_inputs(shape, 11)
+    np.testing.assert_allclose(O.attn_mode(mode, shape, x), _torch_pipeline(shape, x, mode), rtol=1e-11, atol=1e-12)
+
+
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
+def test_pipeline_nondefault_scale_base_eps_matches_torch_restatement(mode):
+    # explicit softmax scale, RoPE base 10 and LayerNorm epsilon 1e-3 (none of them the defaults)
+    shape = tiny_shape(S=2, H=2, ln_eps=1e-3, softmax_scale=0.2, rope_base=10.0)
+    x = W.make_random_inputs(shape, 12)
     np.testing.assert_allclose(O.attn_mode(mode, shape, x), _torch_pipeline(shape, x, mode), rtol=1e-11, atol=1e-12)
 
 
