@@ -64,10 +64,28 @@ def query_sample(mode, shape, count, seed):
     return W.query_subset(shape.S * shape.T, count, seed)
 
 
+def oracle_rows(mode, shape, inputs, queries, workers=None):
+    """The oracle's rows for ``queries``, computed in query chunks on a thread
+    pool (numpy releases the GIL in its array kernels; each chunk is an
+    independent oracle call, and every query row is independent of the others,
+    so the result equals one call on all queries)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
+    queries = np.asarray(queries, dtype=np.int64)
+    workers = workers or os.cpu_count() or 1
+    if len(queries) < 4096 or workers == 1:
+        return O.attn_mode(mode, shape, inputs, queries)
+    chunks = np.array_split(queries, 2 * workers)
+    with threadpool_limits(1), ThreadPoolExecutor(workers) as ex:
+        parts = list(ex.map(lambda c: O.attn_mode(mode, shape, inputs, c), chunks))
+    return np.concatenate(parts, axis=0)
+
+
 def check_mode(mode, shape, inputs, count=None, seed=0, out=None):
     """Run the GPU path, compare ``count`` sampled queries (all when None)."""
     out = run_gpu(mode, shape, inputs, out=out)
     q = query_sample(mode, shape, count if count is not None else 1 << 62, seed)
-    want = O.attn_mode(mode, shape, inputs, q)
+    want = oracle_rows(mode, shape, inputs, q)
     got = rows(out, shape, q)
     return assert_close(got, want, f"{mode} {shape}"), out
