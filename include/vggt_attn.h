@@ -167,8 +167,13 @@ int vggt_attn_abi_version(void);
  *     Global mode fits up to S*T*H ~ 262,000 token-heads (e.g. 15 frames of
  *     1031 tokens x 16 heads); register mode up to S*n_special*H ~ 174,000.
  *   - The first call on a device looks up the scratch array's device address
- *     (cudaGetSymbolAddress, with that device current) and caches it; make that
- *     first call before any stream capture on the device.
+ *     (cudaGetSymbolAddress, with that device current) and caches it together
+ *     with the id of the CUDA context it belongs to; make that first call
+ *     before any stream capture on the device.  A device reset
+ *     (cudaDeviceReset) unloads the library's module with the context: the
+ *     cached address is then invalid, and the first call in the new context
+ *     looks it up again (so, after a reset, that call too should come before
+ *     any stream capture).
  *   - All calls share the one array, and it keeps the last call's contents
  *     (the prologue clears the status word each call; everything else is fully
  *     rewritten before it is read).  Calls that may overlap on the GPU -- on

@@ -455,28 +455,66 @@ int vggt_attn_abi_version(void) { return VGGT_ATTN_ABI_VERSION; }
 // not call cudaMalloc/cudaFree, fixed device-memory budgets): the workspace is
 // this file-scope array, which every GPU that loads the library holds until
 // the process exits.  In host code `noalloc_scratch` names a host-side stand-in,
-// not the device memory, so its device address is looked up once per device
-// with cudaGetSymbolAddress and only that address is passed to the kernels.
+// not the device memory, so its device address is looked up with
+// cudaGetSymbolAddress (with the device current) and only that address is
+// passed to the kernels.
 namespace {
 
 static __device__ __align__(256) unsigned char noalloc_scratch[VGGT_ATTN_NOALLOC_SCRATCH_BYTES];
 
 constexpr int kMaxDevices = 64;
 std::mutex noalloc_mutex;
-void* noalloc_ptr[kMaxDevices] = {};
+// Per device: the address and the CUDA context it belongs to.  A device reset
+// (cudaDeviceReset) destroys the primary context and with it the module that
+// holds the array; the next runtime call creates a new context with a new id,
+// so the address is looked up again instead of reusing a dangling one.
+struct NoallocSlot {
+  unsigned long long ctx_id;
+  void* ptr;
+};
+NoallocSlot noalloc_slot[kMaxDevices] = {};
 
-// Device address of the scratch array on the current device (set-up on the
-// first call per device, with that device current).
+using PfnCtxGetCurrent = CUresult (*)(CUcontext*);
+using PfnCtxGetId = CUresult (*)(CUcontext, unsigned long long*);
+
+// Id of the calling thread's current context (0 if it cannot be read).
+unsigned long long current_context_id() {
+  static PfnCtxGetCurrent get_current = nullptr;
+  static PfnCtxGetId get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<PfnCtxGetCurrent>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetId", &p, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PfnCtxGetId>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_current || !get_id || get_current(&ctx) != CUDA_SUCCESS || !ctx || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device, looked up the
+// first time a context of that device calls (set-up), with that device current.
 int noalloc_scratch_address(void** ptr) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return VGGT_ATTN_ERR_CUDA;
   std::lock_guard<std::mutex> lock(noalloc_mutex);
-  if (!noalloc_ptr[dev]) {
+  NoallocSlot& slot = noalloc_slot[dev];
+  const unsigned long long ctx = current_context_id();   // 0 before the runtime has made a context current
+  if (!slot.ptr || ctx == 0 || slot.ctx_id != ctx) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, noalloc_scratch) != cudaSuccess || p == nullptr) return VGGT_ATTN_ERR_CUDA;
-    noalloc_ptr[dev] = p;
+    slot.ptr = p;
+    slot.ctx_id = current_context_id();                   // the context the lookup ran in
   }
-  *ptr = noalloc_ptr[dev];
+  *ptr = slot.ptr;
   return VGGT_ATTN_OK;
 }
 
