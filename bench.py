@@ -231,12 +231,15 @@ def oracle_sample(workload, n_queries: int, seed: int = 0):
     return dt, flops, threads
 
 
-def headline_config(w, extra=None):
+def headline_config(w, world: int = 1):
+    """The `config` of the JSON line; both arms (ours and --impl reference) print this same object."""
     shape = w.shape
-    cfg = {"workload": w.name, "mode": "global", "frames": shape.S, "tokens": shape.S * shape.T,
-           "heads": shape.H, "head_dim": 64, "flops_per_step_per_gpu": attention_flops("global", shape)}
-    cfg.update(extra or {})
-    return cfg
+    qkv_mb = shape.S * shape.T * 3 * shape.H * 64 * 2 / 1e6
+    ws_mb = 2 * shape.S * shape.T * shape.H * 64 * 2 / 1e6
+    return {"workload": w.name, "mode": "global", "frames": shape.S, "tokens": shape.S * shape.T,
+            "heads": shape.H, "head_dim": 64, "flops_per_step_per_gpu": attention_flops("global", shape),
+            "l2": f"no flush: qkv {qkv_mb:.0f} MB + workspace {ws_mb:.0f} MB read per step exceed the 126 MB L2",
+            "parallelism": f"independent replicas x{world} (weak)"}
 
 
 def cpu_baseline(n_queries: int):
@@ -245,7 +248,7 @@ def cpu_baseline(n_queries: int):
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": threads, "kind": "oracle",
             "sample": f"fp64 numpy oracle, global mode, {n_queries} seeded queries x all 16 heads over all "
                       f"{w.shape.S * w.shape.T} keys (incl. LN+RoPE of every key), {dt:.1f} s",
-            "seconds": dt}
+            "seconds": dt, "queries": n_queries}
 
 
 def run_reference(args):
@@ -263,9 +266,10 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000 * statistics.mean(times),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "config": headline_config(w, {"sample_queries_per_step": n_q}),
+            "data": "synthetic", "config": headline_config(w, world),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
-                             "sample": f"{n_q} seeded queries x 16 heads over all keys per step"},
+                             "sample": f"{n_q} seeded queries x 16 heads over all keys per step (QK-LayerNorm + "
+                                       "RoPE of every key included), scaled by algorithmic flops"},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -400,22 +404,30 @@ def run_ours(args):
            "serial_ms_per_step": serial_ms}
     del h_qkv, h_out, pws
 
-    # ---- ms/layer per mode on the other workloads (device-drawn inputs of the same shapes)
-    modes = {}
+    roofline["frac_clock_normalised"] = clock_normalised_frac(core_tflops, sm_mhz, peaks)
+    roofline["clock_note"] = ("frac_clock_normalised = (achieved / this run's median SM MHz) / (sustained peak / "
+                              "the SM MHz sampled under load while that peak was measured)")
+
+    # ---- every benchmark configuration: ms/call, the core's TFLOP/s and roofline fraction
+    per_config = []
     if not args.no_modes:
-        modes = mode_timings(V, device, stream)
-    blocks = {}
+        headline = {"call_ms": ms / args.steps, "core_ms": core_ms, "prologue_ms": pro_ms, "sm_mhz": sm_mhz}
+        per_config, cfg_clk = config_timings(V, device, stream, peaks, headline)
+        roofline["per_config"] = per_config
+        roofline["per_config_clocks"] = {k: cfg_clk.get(k) for k in ("sm_mhz", "reasons", "power_w_max")}
+    side = {}
     if not args.no_blocks:
-        blocks = block_timings(V, device, stream)
-        blocks["transformer"] = transformer_timings(V, device, stream)
-    sga, sharded = {}, {}
+        side["blocks"] = block_timings(V, device, stream)
+        side["blocks"]["transformer"] = transformer_timings(V, device, stream)
     if not args.no_modes:
-        sga = sga_timings(V, device, stream, qkv, prm, out, ms / args.steps)
-        sharded = sharded_timings(V, device, stream, qkv, prm, ms / args.steps)
+        side["sga"] = sga_timings(V, device, stream, qkv, prm, out, ms / args.steps)
+        side["sharded_global"] = sharded_timings(V, device, stream, qkv, prm, ms / args.steps)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline(args.cpu_queries)
+        if per_config:
+            cpu["per_config"] = oracle_config_timings(cpu)
 
     if world > 1:
         dist.barrier(device_ids=[device.index])
@@ -425,13 +437,11 @@ def run_ours(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": headline_config(w, {
-                "l2": f"no flush: qkv {qkv.numel() * 2 / 1e6:.0f} MB + workspace {ws_bytes / 1e6:.0f} MB read per "
-                      "step exceed the 126 MB L2",
-                "parallelism": f"independent replicas x{world} (weak)"}),
+            "config": headline_config(w, world),
             "pct_of_peak": 100.0 * value / world / peak,
-            "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "modes": modes,
-            "blocks": blocks, "sga": sga, "sharded_global": sharded, "cpu_baseline": cpu}
+            "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu}
+    if side:   # side measurements (blocks, subsampled and sharded forms) on a line of their own, before the result
+        print(json.dumps({"side_measurements": side}), flush=True)
     print(json.dumps(line), flush=True)
     return 0
 
@@ -658,36 +668,178 @@ def transformer_timings(V, device, stream):
     return res
 
 
-def mode_timings(V, device, stream):
-    """ms per call for each mode on its workload, plus the S=500 layer (register + frame)."""
+# The benchmark's configurations: (label, workload index, mode).  Workload 3 is the headline, timed above.
+CONFIG_RUNS = [("cfg0_global_S2_T69_H4", 0, "global"), ("cfg1_frame_S24", 1, "frame"),
+               ("cfg2_global_S24_N24744", 2, "global"), ("cfg3_global_S100_N103100", 3, "global"),
+               ("cfg4a_register_S500", 4, "register"), ("cfg4b_frame_S500", 4, "frame")]
+
+
+def clock_normalised_frac(tflops, run_mhz, peaks):
+    """Achieved TFLOP/s per MHz of the run's median SM clock, over the sustained GEMM peak per MHz of the
+    clock sampled under load while that peak was measured (None without both clocks)."""
+    peak_mhz = ((peaks.get("clocks_under_load") or {}).get("sm_mhz_median"))
+    peak = peaks.get("bf16_tflops_sustained")
+    if not run_mhz or not peak_mhz or not peak:
+        return None
+    return (tflops / run_mhz) / (peak / peak_mhz)
+
+
+def config_timings(V, device, stream, peaks, headline):
+    """ms per call (QK-norm/RoPE prologue + attention core), the core and the prologue alone, and the
+    core's roofline fraction, for every benchmark configuration; the S=500 layer (register + frame call).
+    Inputs are drawn on the device with the workload's shape and value distribution (timing only; the
+    seeded host inputs are the parity tests' business).  Configs whose inputs fit in L2 (the tiny one)
+    are timed back to back, as a latency figure."""
     import torch
-    res = {}
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    burst = peaks.get("bf16_tflops", peak)
     g = torch.Generator(device=device)
     g.manual_seed(1234)
-    for label, idx, mode in (("frame_S24_T1031", 1, "frame"), ("global_S24_N24744", 2, "global"),
-                             ("register_S500", 4, "register"), ("frame_S500", 4, "frame")):
-        shape = W.workload(idx).shape
-        if label == "frame_S500":
-            pass  # reuses the S=500 tensors of the register entry
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    rows, cache = [], {}
+    for label, idx, mode in CONFIG_RUNS:
+        w = W.workload(idx)
+        shape = w.shape
+        if idx == 3:
+            call_ms, core_ms, pro_ms = headline["call_ms"], headline["core_ms"], headline["prologue_ms"]
         else:
-            qkv = torch.randn((shape.S, shape.T, 3, shape.H, 64), generator=g, device=device,
-                              dtype=torch.float32).to(torch.bfloat16)
-            prm = {k: (1.0 if "gamma" in k else 0.0) + 0.1 * torch.randn((shape.H, 64), generator=g, device=device)
-                   for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}
-            out = torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device=device)
-        wsb = V.vggt_attn_workspace_size(shape, mode)
-        ws = torch.empty(wsb, dtype=torch.uint8, device=device)
-        fn = lambda: V.attend(mode, shape, qkv, prm["q_gamma"], prm["q_beta"], prm["k_gamma"], prm["k_beta"], out,
-                              ws, stream)
-        for _ in range(3):
-            fn()
-        ms = cuda_time_ms(fn, stream, 10)
-        assert V.vggt_attn_read_status(ws, stream) == 0
+            if idx not in cache:
+                cache.clear()
+                qkv = torch.randn((shape.S, shape.T, 3, shape.H, 64), generator=g, device=device,
+                                  dtype=torch.float32).to(torch.bfloat16)
+                prm = [(1.0 if k % 2 == 0 else 0.0) + 0.1 * torch.randn((shape.H, 64), generator=g, device=device)
+                       for k in range(4)]
+                cache[idx] = (qkv, prm, torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16,
+                                                    device=device))
+            qkv, prm, out = cache[idx]
+            wsb = V.vggt_attn_workspace_size(shape, mode)
+            ws = torch.empty(wsb, dtype=torch.uint8, device=device)
+            call = lambda: V.attend(mode, shape, qkv, *prm, out, ws, stream)  # noqa: E731
+            for _ in range(3):
+                call()
+            iters = 200 if idx == 0 else 20
+            call_ms = cuda_time_ms(call, stream, iters)
+            core_ms = cuda_time_ms(lambda: V.vggt_attn_core(mode, shape, qkv, out, ws, wsb, stream), stream, iters)
+            pro_ms = cuda_time_ms(lambda: V.vggt_attn_prologue(mode, shape, qkv, *prm, ws, wsb, stream), stream,
+                                  iters)
+            assert V.vggt_attn_read_status(ws, stream) == 0
+            del ws
         f = attention_flops(mode, shape)
-        res[label] = {"ms": ms, "tflops": f / (ms / 1000) / 1e12, "gbs_min_io": io_bytes(mode, shape) / (ms / 1000) / 1e9}
-        del ws
-    res["layer_S500_register_plus_frame_ms"] = res["register_S500"]["ms"] + res["frame_S500"]["ms"]
+        core_tf = f / (core_ms / 1000) / 1e12
+        row = {"config": label, "mode": mode, "ms": call_ms, "core_ms": core_ms, "prologue_ms": pro_ms,
+               "tflops": f / (call_ms / 1000) / 1e12, "core_tflops": core_tf, "frac": core_tf / peak,
+               "frac_burst": core_tf / burst,
+               "prologue_hbm_gbs": io_bytes(mode, shape) / (pro_ms / 1000) / 1e9}
+        if mode == "register":
+            row["gbs_min_io"] = io_bytes(mode, shape) / (call_ms / 1000) / 1e9
+        rows.append(row)
+    cache.clear()
+    clk = clocks.stop()
+    mhz = clk.get("sm_mhz")
+    for row in rows:
+        run_mhz = headline["sm_mhz"] if row["config"].startswith("cfg3") else mhz
+        row["frac_clock_normalised"] = clock_normalised_frac(row["core_tflops"], run_mhz, peaks)
+        row["sm_mhz"] = run_mhz
+    by = {r["config"]: r for r in rows}
+    layer = by["cfg4a_register_S500"]["ms"] + by["cfg4b_frame_S500"]["ms"]
+    rows.append({"config": "cfg4_layer_S500_register_plus_frame", "mode": "layer", "ms": layer,
+                 "tflops": (attention_flops("register", W.workload(4).shape) +
+                            attention_flops("frame", W.workload(4).shape)) / (layer / 1000) / 1e12})
+    return rows, clk
+
+
+def oracle_config_timings(headline_cpu):
+    """The fp64 oracle timed on this host for every configuration: in full where that takes seconds, else on a
+    seeded sample with the full time extrapolated by the ratio of algorithmic work (labelled)."""
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    res = []
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    def entry(label, mode, shape, sample, seconds, frac_of_work):
+        full = seconds / frac_of_work
+        return {"config": label, "mode": mode, "sample": sample, "seconds": seconds, "full_seconds": full,
+                "extrapolated": frac_of_work < 1.0, "tflops": attention_flops(mode, shape) / full / 1e12,
+                "cores": threads}
+
+    for label, idx, mode in CONFIG_RUNS:
+        w = W.workload(idx)
+        shape = w.shape
+        if idx == 3:
+            res.append(entry(label, mode, shape, headline_cpu["sample"], headline_cpu["seconds"],
+                             headline_cpu["queries"] / (shape.S * shape.T)))
+            continue
+        x = _ORACLE_INPUTS.get(w.name)
+        if x is None:
+            x = _ORACLE_INPUTS.setdefault(w.name, W.make_inputs(w))
+        if mode == "global" and idx == 2:
+            q = W.query_subset(shape.S * shape.T, 1024, w.seed)
+            dt = timed(lambda: O.attn_global(shape, x, q))
+            res.append(entry(label, mode, shape, "1024 seeded queries x 16 heads over all 24,744 keys", dt,
+                             1024 / (shape.S * shape.T)))
+        elif mode == "frame" and idx == 4:
+            frames = np.sort(np.random.default_rng([w.seed, 5]).choice(shape.S, 4, replace=False))
+            q = (frames[:, None] * shape.T + np.arange(shape.T)[None, :]).reshape(-1)
+            dt = timed(lambda: O.attn_frame(shape, x, q))
+            res.append(entry(label, mode, shape, "every query of 4 seeded frames (of 500)", dt, 4 / shape.S))
+        else:
+            dt = timed(lambda: O.attn_mode(mode, shape, x))
+            res.append(entry(label, mode, shape, "full", dt, 1.0))
+    _ORACLE_INPUTS.clear()
     return res
+
+
+def run_one(args) -> int:
+    """One attention mode (or one transformer block, or subsampled / descriptor global attention) on
+    device-drawn inputs of a workload's shape: one warm-up call, then --calls timed calls; prints ms per call.
+    A small driver for profiling a single kernel under ncu (no side measurements, no oracle)."""
+    import torch
+    import vit_attention_b200 as V
+    mode = args.one
+    torch.cuda.set_device(0)
+    shape = W.workload(args.workload).shape
+    if args.frames > 0:
+        shape = dataclasses.replace(shape, S=args.frames)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1234)
+    H, C = shape.H, shape.H * 64
+    if args.block:
+        w = random_block_weights(H, g, torch.device("cuda"))
+        x = torch.randn((shape.S * shape.T, C), generator=g, device="cuda").to(torch.bfloat16)
+        ws = torch.empty(V.vggt_block_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+
+        def call():
+            V.vggt_block_forward(mode, shape, x, w, 1e-6, ws)
+    else:
+        qkv = torch.randn((shape.S, shape.T, 3, H, 64), generator=g, device="cuda").to(torch.bfloat16)
+        prm = [(1.0 if k % 2 == 0 else 0.0) + 0.1 * torch.randn((H, 64), generator=g, device="cuda")
+               for k in range(4)]
+        out = torch.empty((shape.S, shape.T, H, 64), dtype=torch.bfloat16, device="cuda")
+        if args.sga or args.desc:
+            sz = args.sga or args.desc
+            fn = V.vggt_attn_global_sga if args.sga else V.vggt_attn_global_desc
+            ws = torch.empty(V.vggt_attn_sga_workspace_size(shape, sz, sz), dtype=torch.uint8, device="cuda")
+
+            def call():
+                fn(shape, sz, sz, qkv, *prm, out, ws)
+        else:
+            ws = torch.empty(V.vggt_attn_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+
+            def call():
+                V.attend(mode, shape, qkv, *prm, out, ws)
+    call()
+    torch.cuda.synchronize()
+    ms = cuda_time_ms(call, torch.cuda.current_stream(), max(args.calls, 1))
+    status = V.vggt_attn_read_status(ws)
+    print(json.dumps({"one": mode, "block": args.block, "sga": args.sga, "desc": args.desc, "S": shape.S,
+                      "T": shape.T, "H": H, "ms_per_call": ms, "status": status}), flush=True)
+    return 0 if status == 0 else 1
 
 
 def main():
@@ -705,9 +857,19 @@ def main():
     ap.add_argument("--linear-only", default=None, metavar="M,N,K",
                     help="run vggt_linear on an M x N x K problem a few times and exit (a small case for ncu)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--one", choices=("frame", "global", "register"), default=None,
+                    help="run only this mode on --workload's shape (--frames, --calls, --block, --sga, --desc) and "
+                         "exit: a small case for ncu")
+    ap.add_argument("--frames", type=int, default=0, help="with --one: override the frame count S")
+    ap.add_argument("--calls", type=int, default=3, help="with --one: timed calls after one warm-up call")
+    ap.add_argument("--block", action="store_true", help="with --one: a whole transformer block")
+    ap.add_argument("--sga", type=int, default=0, help="with --one global: subsampled global attention, s x s grid")
+    ap.add_argument("--desc", type=int, default=0, help="with --one global: descriptor attention, s x s windows")
     args = ap.parse_args()
     if args.linear_only:
         return linear_only(args.linear_only)
+    if args.one:
+        return run_one(args)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
