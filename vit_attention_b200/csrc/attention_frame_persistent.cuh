@@ -7,10 +7,14 @@
 // each CTA (two per SM, 256 threads, 256 TMEM columns) walks the units
 // u = blockIdx.x, blockIdx.x + gridDim.x, ... (unit = one 128-query tile of
 // one (frame, head), tiles of a problem consecutive) and keeps its pipeline
-// running across units: the producer loads the next unit's Q into a second
-// buffer and its K/V into the same ring, the softmax warps copy the next Q
-// into TMEM as soon as the current unit's last QK^T product has completed,
-// so the next unit's first products run during this unit's epilogue.  The
+// running across units: the producer loads the next unit's Q into the one Q
+// buffer as soon as the current Q is in TMEM (a unit ahead of its use) and its
+// K/V into the same ring, the softmax warps copy the next Q into TMEM as soon
+// as the current unit's last QK^T product has completed, so the next unit's
+// first products run during this unit's epilogue.  The epilogue writes the
+// output tile through a shared-memory staging tile with one TMA store (rows
+// past the frame's end are clipped by the tensor map); a thread's 128-byte
+// output row would otherwise be a global store to a line of its own.  The
 // per-step work is that of attn_core_kernel (see attention_sm100.cuh) -- Q in
 // TMEM, two S buffers, online softmax with a lazily moved reference max --
 // with two differences that fit the 256 TMEM columns of a CTA that shares its
@@ -37,14 +41,15 @@ constexpr int KV_BYTES = BN * D * 2;                    // 10 KB key or value ti
 constexpr uint32_t IDESC_QK = idesc_bf16_f32(BM, BN, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16_f32(BM, D, 0, 1);   // V is MN-major
 constexpr int STAGES = 4;
-constexpr int OFF_Q = 0;                                // two Q buffers
-constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
+constexpr int OFF_Q = 0;                                // one Q buffer
+constexpr int OFF_STG = OFF_Q + Q_BYTES;                // output staging tile (128 rows x 128 B)
+constexpr int OFF_K = OFF_STG + Q_BYTES;
 constexpr int OFF_V = OFF_K + STAGES * KV_BYTES;
 constexpr int OFF_BAR = OFF_V + STAGES * KV_BYTES;
 enum {
-  BAR_Q_FULL = 0,                       // [Q buffer]
-  BAR_Q_EMPTY = BAR_Q_FULL + 2,         // [Q buffer]
-  BAR_KV_FULL = BAR_Q_EMPTY + 2,
+  BAR_Q_FULL = 0,
+  BAR_Q_EMPTY = BAR_Q_FULL + 1,
+  BAR_KV_FULL = BAR_Q_EMPTY + 1,
   BAR_KV_EMPTY = BAR_KV_FULL + STAGES,
   BAR_S_FULL = BAR_KV_EMPTY + STAGES,   // [buffer]
   BAR_P_FULL = BAR_S_FULL + 2,          // [buffer]
@@ -106,8 +111,8 @@ __device__ __forceinline__ void mbar_arrive_count(uint32_t bar, uint32_t count) 
 
 // Softmax warpgroup (warps 4-7): thread r owns query row r of every unit.
 __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const FrameUnits& fu, const uint8_t* smem,
-                                                   uint32_t tmem, uint32_t bar0, volatile int* abort_flag, int n_kv,
-                                                   int warp, int lane) {
+                                                   const CUtensorMap& tmap_o, uint32_t tmem, uint32_t bar0,
+                                                   volatile int* abort_flag, int n_kv, int warp, int lane) {
   using namespace fp;
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   const int quarter = warp & 3;
@@ -118,13 +123,13 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
   const PolyConsts pc = poly_consts();
   const bool leader = (threadIdx.x & 127) == 0;
 
-  // Q tile of local unit i (buffer i % 2, 128-byte swizzle) -> TMEM columns
+  // Q tile of local unit i (128-byte swizzle) -> TMEM columns
   // COL_Q.. (row r in lane r, dims (2c, 2c+1) in column c).
   auto copy_q = [&](int i) -> bool {
-    bool ok = wait_bounded(bar(BAR_Q_FULL + (i & 1)), (i >> 1) & 1, abort_flag, p.status, p.timeout_ns, 0x630u);
+    bool ok = wait_bounded(bar(BAR_Q_FULL), i & 1, abort_flag, p.status, p.timeout_ns, 0x630u);
     ok = __all_sync(0xffffffffu, ok);
     if (!ok) return false;
-    const uint4* qrow = reinterpret_cast<const uint4*>(smem + OFF_Q + (i & 1) * Q_BYTES + row * 128);
+    const uint4* qrow = reinterpret_cast<const uint4*>(smem + OFF_Q + row * 128);
     uint32_t qr[32];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
@@ -138,7 +143,7 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bar(BAR_Q_TMEM));
-    mbar_arrive(bar(BAR_Q_EMPTY + (i & 1)));
+    mbar_arrive(bar(BAR_Q_EMPTY));
     return true;
   };
 
@@ -263,12 +268,14 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
     tmem_wait_ld();
     tc_fence_before();
     mbar_arrive(bar(BAR_O_FREE));
-    const int qi = q0 + row;
-    if (qi < p.L) {
+    // Output tile: each row into the staging tile (128-byte swizzle), then one
+    // TMA store of the tile (rows past the frame's end are clipped by the map).
+    {
+      const bool issuer = (threadIdx.x & 127) == 0;
+      if (issuer) bulk_wait_read_all();            // the previous unit's store has read the staging tile
+      named_bar_sync(1, 128);
       const float inv = 1.f / l_run;
-      const long long out_row = static_cast<long long>(b) * p.out_T +
-                                static_cast<long long>(qi / p.out_group) * p.out_T + (qi % p.out_group);
-      uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D);
+      uint4* srow = reinterpret_cast<uint4*>(const_cast<uint8_t*>(smem) + OFF_STG + row * 128);
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
 #pragma unroll
@@ -279,20 +286,28 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
           w.y = pack_bf16x2(__uint_as_float(o[2]) * inv, __uint_as_float(o[3]) * inv);
           w.z = pack_bf16x2(__uint_as_float(o[4]) * inv, __uint_as_float(o[5]) * inv);
           w.w = pack_bf16x2(__uint_as_float(o[6]) * inv, __uint_as_float(o[7]) * inv);
-          dst[c * 4 + v] = w;
+          srow[(c * 4 + v) ^ (row & 7)] = w;
         }
+      }
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      named_bar_sync(1, 128);
+      if (issuer) {
+        tma_store_4d(&tmap_o, smem_addr(smem) + OFF_STG, 0, h, q0, b);
+        bulk_commit();
       }
     }
     G += n_kv;
   }
+  if ((threadIdx.x & 127) == 0) bulk_wait_all();
 }
 
 // Grid: min(n_units, 2 x SMs) CTAs, one dimension.  The producer runs ahead
 // of the softmax by up to one unit of Q and STAGES key steps of K/V.
+// tmap_o: out[S][T][H][64] as (dim, head, token, frame), box 64 x 1 x 128 x 1.
 __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
     attn_frame_persistent_kernel(const __grid_constant__ CUtensorMap tmap_q, const __grid_constant__ CUtensorMap tmap_k,
-                                 const __grid_constant__ CUtensorMap tmap_v, const CoreParams p,
-                                 const FrameUnits fu) {
+                                 const __grid_constant__ CUtensorMap tmap_v, const __grid_constant__ CUtensorMap tmap_o,
+                                 const CoreParams p, const FrameUnits fu) {
   using namespace fp;
   using core::NV;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -311,10 +326,8 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
   const int n_kv = (p.Lk + BN - 1) / BN;
 
   if (threadIdx.x == 0) {
-    for (int qb = 0; qb < 2; ++qb) {
-      mbar_init(bar(BAR_Q_FULL + qb), 1);
-      mbar_init(bar(BAR_Q_EMPTY + qb), 128);
-    }
+    mbar_init(bar(BAR_Q_FULL), 1);
+    mbar_init(bar(BAR_Q_EMPTY), 128);
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar(BAR_KV_FULL + s), 1);
       mbar_init(bar(BAR_KV_EMPTY + s), 1);
@@ -333,6 +346,7 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
     tma_prefetch_desc(&tmap_q);
     tma_prefetch_desc(&tmap_k);
     tma_prefetch_desc(&tmap_v);
+    tma_prefetch_desc(&tmap_o);
   }
   if (warp == 1) {
     tmem_alloc(smem_addr(const_cast<uint32_t*>(tmem_slot)), TMEM_COLS);
@@ -346,7 +360,7 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
 
   if (warp >= 4) {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REGS_SOFTMAX));
-    if (!skip) frame_softmax_role(p, fu, smem, tmem, bar0, abort_flag, n_kv, warp, lane);
+    if (!skip) frame_softmax_role(p, fu, smem, tmap_o, tmem, bar0, abort_flag, n_kv, warp, lane);
   } else {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REGS_PRODUCER));
   }
@@ -355,21 +369,20 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
     if (lane == 0 && !skip) {
       int kv_issued[STAGES];
       for (int s = 0; s < STAGES; ++s) kv_issued[s] = 0;
-      int q_issued[2] = {0, 0};
+      int q_issued = 0;
       bool ok = true;
       for (int i = 0; ok; ++i) {
         const int u = static_cast<int>(blockIdx.x) + i * static_cast<int>(gridDim.x);
         if (u >= fu.n_units) break;
         int q0, h, b;
         frame_unit(p, fu, u, q0, h, b);
-        const int qb = i & 1;
-        if (i >= 2) {
-          ok = wait_bounded(bar(BAR_Q_EMPTY + qb), ((i >> 1) - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x580u);
+        if (i >= 1) {   // unit i-1's Q has been copied into TMEM
+          ok = wait_bounded(bar(BAR_Q_EMPTY), (i - 1) & 1, abort_flag, p.status, p.timeout_ns, 0x580u);
           if (!ok) break;
         }
-        mbar_arrive_expect_tx(bar(BAR_Q_FULL + qb), Q_BYTES);
-        tma_load_3d(sbase + OFF_Q + qb * Q_BYTES, &tmap_q, bar(BAR_Q_FULL + qb), 0, q0, h * p.B + b);
-        ++q_issued[qb];
+        mbar_arrive_expect_tx(bar(BAR_Q_FULL), Q_BYTES);
+        tma_load_3d(sbase + OFF_Q, &tmap_q, bar(BAR_Q_FULL), 0, q0, h * p.B + b);
+        ++q_issued;
         for (int j = 0; j < n_kv; ++j) {
           const int k = i * n_kv + j;
           const int st = k % STAGES;
@@ -387,8 +400,7 @@ __global__ void __launch_bounds__(fp::THREADS, fp::CTAS_PER_SM)
       if (!ok) {
         // Drain: the last load issued into every stage and Q buffer must land
         // before this CTA's shared memory is released.
-        for (int qb = 0; qb < 2; ++qb)
-          if (q_issued[qb] > 0) wait_drain(bar(BAR_Q_FULL + qb), (q_issued[qb] - 1) & 1, p.timeout_ns);
+        if (q_issued > 0) wait_drain(bar(BAR_Q_FULL), (q_issued - 1) & 1, p.timeout_ns);
         for (int st = 0; st < STAGES; ++st)
           if (kv_issued[st] > 0) wait_drain(bar(BAR_KV_FULL + st), (kv_issued[st] - 1) & 1, p.timeout_ns);
       }

@@ -238,6 +238,15 @@ int launch_core_cfg(const ModeGeometry& g, int H, const CUtensorMap& mq, const C
 // frame) units with a stride of the grid size.
 int launch_frame_persistent(const ModeGeometry& g, int H, const CUtensorMap& mq, const CUtensorMap& mk,
                             const CUtensorMap& mv, const vggt::CoreParams& p, cudaStream_t stream) {
+  // output tile map: out[S][T][H][64] as (dim, head, token, frame), one 128-token box per store
+  CUtensorMap mo;
+  {
+    const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(g.L),
+                                static_cast<cuuint64_t>(g.B)};
+    const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(H) * 128 * g.L};
+    const cuuint32_t box[4] = {64, 1, vggt::core::BM, 1};
+    if (!make_map(&mo, p.out, 4, dims, strides, box)) return VGGT_ATTN_ERR_CUDA;
+  }
   if (cudaFuncSetAttribute(vggt::attn_frame_persistent_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            vggt::fp::SMEM_ALLOC) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
@@ -256,7 +265,7 @@ int launch_frame_persistent(const ModeGeometry& g, int H, const CUtensorMap& mq,
   long long grid = static_cast<long long>(sms) * vggt::fp::CTAS_PER_SM;
   if (grid > n_units) grid = n_units;
   vggt::attn_frame_persistent_kernel<<<static_cast<unsigned>(grid), vggt::fp::THREADS, vggt::fp::SMEM_ALLOC,
-                                       stream>>>(mq, mk, mv, p, fu);
+                                       stream>>>(mq, mk, mv, mo, p, fu);
   return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
