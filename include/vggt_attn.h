@@ -73,7 +73,9 @@ enum {
   VGGT_ATTN_ERR_CUDA = -5,              /* a CUDA runtime/driver call or a launch failed */
   VGGT_ATTN_ERR_TIMEOUT = -6,           /* a bounded wait inside a kernel expired (vggt_attn_read_status) */
   VGGT_ATTN_ERR_UNSUPPORTED_DEVICE = -7, /* current device is not compute capability 10.0 (sm_100a) */
-  VGGT_ATTN_ERR_SCRATCH_TOO_SMALL = -8   /* vggt_attn_noalloc: the problem needs more than VGGT_ATTN_NOALLOC_SCRATCH_BYTES */
+  VGGT_ATTN_ERR_SCRATCH_TOO_SMALL = -8,  /* vggt_attn_noalloc: the problem needs more than VGGT_ATTN_NOALLOC_SCRATCH_BYTES */
+  VGGT_ATTN_ERR_BOUNDS = -9              /* debug build only (libvggt_attn_debug.so, -DVGGT_DEBUG): a device-side
+                                            bounds check failed; the access was skipped, the status word records it */
 };
 
 /* Attention modes. */

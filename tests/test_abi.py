@@ -30,6 +30,17 @@ def declared_functions():
     return sorted(set(names))
 
 
+def test_debug_build_exports_every_declared_function(V):
+    import __graft_entry__
+    lib_path = __graft_entry__._build_module().build(debug=True)
+    assert lib_path.endswith("libvggt_attn_debug.so")
+    lib = ctypes.CDLL(lib_path)
+    for n in declared_functions():
+        assert hasattr(lib, n), n
+    lib.vggt_attn_error_string.restype = ctypes.c_char_p
+    assert b"bounds check" in lib.vggt_attn_error_string(V.ERR_BOUNDS)
+
+
 def test_library_exports_every_declared_function(V):
     names = declared_functions()
     assert len(names) >= 10

@@ -13,7 +13,9 @@ import ctypes
 import os
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libvggt_attn.so")
+# VGGT_ATTN_LIBRARY=debug loads the debug build (device-side bounds checks, `build.py --debug`) instead.
+LIB_PATH = os.path.join(_HERE, "libvggt_attn_debug.so" if os.environ.get("VGGT_ATTN_LIBRARY") == "debug"
+                        else "libvggt_attn.so")
 
 FRAME, GLOBAL, REGISTER = 0, 1, 2
 MODES = {"frame": FRAME, "global": GLOBAL, "register": REGISTER}
@@ -27,6 +29,7 @@ ERR_CUDA = -5
 ERR_TIMEOUT = -6
 ERR_UNSUPPORTED_DEVICE = -7
 ERR_SCRATCH_TOO_SMALL = -8
+ERR_BOUNDS = -9
 NOALLOC_SCRATCH_BYTES = 64 << 20
 
 

@@ -1,6 +1,6 @@
 """Build libvggt_attn.so in-tree for sm_100a (B200).
 
-    python vit_attention_b200/build.py [--force]
+    python vit_attention_b200/build.py [--force] [--debug]
 
 (Run as a file, not through the package: the package's __init__ loads the
 library this script builds.)
@@ -18,6 +18,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libvggt_attn.so")
+LIB_DEBUG = os.path.join(HERE, "libvggt_attn_debug.so")   # -DVGGT_DEBUG: device-side bounds checks
 SOURCES = [os.path.join(HERE, "csrc", "vggt_attn.cu")]
 DEPENDS = SOURCES + sorted(os.path.join(HERE, "csrc", f) for f in os.listdir(os.path.join(HERE, "csrc"))
                            if f.endswith(".cuh")) + [os.path.join(ROOT, "include", "vggt_attn.h")]
@@ -31,26 +32,30 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found (set NVCC or put the CUDA 12.9 toolkit on PATH)")
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(f) <= t for f in DEPENDS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Build the release library, or with debug=True the debug build (libvggt_attn_debug.so: -DVGGT_DEBUG,
+    device-side bounds checks that record VGGT_ATTN_ERR_BOUNDS instead of faulting)."""
+    lib = LIB_DEBUG if debug else LIB
+    if not force and up_to_date(lib):
+        return lib
     cmd = [nvcc(), *ARCH_FLAGS, "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-           "-Xptxas", "-v", "-I", os.path.join(ROOT, "include"), "-o", LIB + ".tmp", *SOURCES]
+           "-Xptxas", "-v", "-I", os.path.join(ROOT, "include"), *(["-DVGGT_DEBUG"] if debug else []),
+           "-o", lib + ".tmp", *SOURCES]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stderr}")
     if verbose:
         sys.stderr.write(res.stderr)
-    os.replace(LIB + ".tmp", LIB)
-    return LIB
+    os.replace(lib + ".tmp", lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose=True))
+    print(build(force="--force" in sys.argv, verbose=True, debug="--debug" in sys.argv))

@@ -291,7 +291,7 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
       }
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
       named_bar_sync(1, 128);
-      if (issuer) {
+      if (issuer && VGGT_DBG_BOUNDS(h < p.H && q0 < p.L && b < p.B, p.status, 0x910u)) {
         tma_store_4d(&tmap_o, smem_addr(smem) + OFF_STG, 0, h, q0, b);
         bulk_commit();
       }

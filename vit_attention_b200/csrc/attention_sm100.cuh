@@ -91,6 +91,7 @@ struct CoreParams {
   int out_T;          // tokens per frame of `out`
   int out_group;      // query i of problem b -> out row b*out_T + (i/out_group)*out_T + i%out_group
   uint16_t* out;      // bf16 [.][H][64]
+  long long out_elems;  // elements of out (bounds of the debug build's checks)
   int* status;
   unsigned long long timeout_ns;
   SgaParams sga;      // SGA configuration only
@@ -503,8 +504,9 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
       const long long out_row = static_cast<long long>(b) * p.out_T +
                                 static_cast<long long>(i / p.out_group) * p.out_T + (i % p.out_group);
       uint4* dst = reinterpret_cast<uint4*>(p.out + (out_row * p.H + h) * D);
+      const bool in_bounds = VGGT_DBG_BOUNDS((out_row * p.H + h + 1) * D <= p.out_elems, p.status, 0x900u);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
+      for (int c = 0; c < 2 && in_bounds; ++c) {
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
           uint4 w;

@@ -23,6 +23,17 @@ __device__ __forceinline__ void record_error(int* status, int code, uint32_t whe
   }
 }
 
+// Device-side bounds checks of the debug build (compiled with -DVGGT_DEBUG):
+// a failed check records VGGT_ATTN_ERR_BOUNDS with the check's tag in the
+// status word and the access it guards is skipped instead of faulting.  In
+// the release build the checks compile to `true`.
+#ifdef VGGT_DEBUG
+#define VGGT_DBG_BOUNDS(cond, status, where) \
+  ((cond) ? true : (::vggt::record_error((status), VGGT_ATTN_ERR_BOUNDS, (where)), false))
+#else
+#define VGGT_DBG_BOUNDS(cond, status, where) true
+#endif
+
 __device__ __forceinline__ bool status_is_set(const int* status) {
   return *reinterpret_cast<const volatile int*>(status) != 0;
 }

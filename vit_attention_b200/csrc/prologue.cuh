@@ -66,6 +66,8 @@ struct PrologueParams {
   int k_token_major;      // k written token-major [L][H][64] (like v) instead of the head planes
   int* status;         // cleared by block 0 when zero_status (the first kernel of a call)
   int zero_status;
+  long long qkv_elems;    // elements of qkv, of each q/k destination and of the v destination
+  long long qk_elems, v_elems;   // (bounds of the debug build's checks)
   int n_tok;              // tokens in the mode's token list (< 2^31, checked on the host)
   int T, H, n_special, grid_h, grid_w;
   int mode;               // VGGT_ATTN_FRAME / GLOBAL / REGISTER
@@ -161,16 +163,22 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
 #pragma unroll
       for (int k = 0; k < TOKENS; ++k) {
         const uint16_t* src = p.qkv + w[k].src + row_src;
-        ra[k] = *reinterpret_cast<const uint4*>(src);
-        rb[k] = *reinterpret_cast<const uint4*>(src + 16);
+        if (VGGT_DBG_BOUNDS(w[k].src + row_src + 24 <= p.qkv_elems, p.status, 0x920u)) {
+          ra[k] = *reinterpret_cast<const uint4*>(src);
+          rb[k] = *reinterpret_cast<const uint4*>(src + 16);
+        } else {
+          ra[k] = rb[k] = make_uint4(0, 0, 0, 0);
+        }
       }
 #pragma unroll
       for (int k = 0; k < TOKENS; ++k) {
         if (i0 + k * static_cast<int>(gridDim.x) >= p.n_tok) continue;
         if (c == 2) {   // register-mode v gather: plain copy
           uint16_t* dst = p.ws_v + w[k].dst_v + h * 64 + base;
-          *reinterpret_cast<uint4*>(dst) = ra[k];
-          *reinterpret_cast<uint4*>(dst + 16) = rb[k];
+          if (VGGT_DBG_BOUNDS(w[k].dst_v + h * 64 + base + 24 <= p.v_elems, p.status, 0x921u)) {
+            *reinterpret_cast<uint4*>(dst) = ra[k];
+            *reinterpret_cast<uint4*>(dst + 16) = rb[k];
+          }
           continue;
         }
         float xa[8], xb[8];
@@ -231,10 +239,13 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
         ob.y = pack_bf16x2(xb[2] * mult, xb[3] * mult);
         ob.z = pack_bf16x2(xb[4] * mult, xb[5] * mult);
         ob.w = pack_bf16x2(xb[6] * mult, xb[7] * mult);
-        uint16_t* dst = (c == 1 && p.k_token_major) ? p.ws_qk[1] + w[k].dst_v + h * 64 + base
-                                                    : p.ws_qk[c] + w[k].dst_qk + row_dst;
-        *reinterpret_cast<uint4*>(dst) = oa;
-        *reinterpret_cast<uint4*>(dst + 16) = ob;
+        const long long dst_off = (c == 1 && p.k_token_major) ? w[k].dst_v + h * 64 + base : w[k].dst_qk + row_dst;
+        uint16_t* dst = p.ws_qk[c] + dst_off;
+        const long long dst_elems = (c == 1 && p.k_token_major) ? p.v_elems : p.qk_elems;
+        if (VGGT_DBG_BOUNDS(dst_off + 24 <= dst_elems, p.status, 0x922u)) {
+          *reinterpret_cast<uint4*>(dst) = oa;
+          *reinterpret_cast<uint4*>(dst + 16) = ob;
+        }
       }
     }
   }

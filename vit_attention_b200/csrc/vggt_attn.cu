@@ -174,6 +174,9 @@ int launch_prologue(int mode, const vggt_attn_shape* s, const void* qkv, const f
   }
   p.status = w.status;
   p.zero_status = clear_status ? 1 : 0;
+  p.qkv_elems = static_cast<long long>(s->S) * s->T * 3 * s->H * 64;
+  p.qk_elems = g.B * g.L * s->H * 64;
+  p.v_elems = g.L * s->H * 64;
   p.n_tok = static_cast<int>(g.n_tok);
   p.T = s->T;
   p.H = s->H;
@@ -307,6 +310,7 @@ int launch_core(int mode, const vggt_attn_shape* s, const void* qkv, void* out, 
   p.out_T = s->T;
   p.out_group = mode == VGGT_ATTN_REGISTER ? s->n_special : static_cast<int>(g.L);
   p.out = static_cast<uint16_t*>(out);
+  p.out_elems = static_cast<long long>(s->S) * s->T * s->H * 64;
   p.status = w.status;
   p.timeout_ns = kDefaultTimeoutNs;
   // Frame mode: one query tile per CTA, two CTAs per SM; global and register
@@ -450,6 +454,7 @@ const char* vggt_attn_error_string(int code) {
     case VGGT_ATTN_ERR_TIMEOUT: return "a bounded wait inside a kernel expired";
     case VGGT_ATTN_ERR_UNSUPPORTED_DEVICE: return "current device is not sm_100 (B200)";
     case VGGT_ATTN_ERR_SCRATCH_TOO_SMALL: return "problem needs more workspace than the fixed 64 MiB scratch of vggt_attn_noalloc";
+    case VGGT_ATTN_ERR_BOUNDS: return "a device-side bounds check of the debug build failed (the access was skipped)";
     default: return "unknown error code";
   }
 }
@@ -925,6 +930,7 @@ extern "C" int vggt_attn_global_sga(const vggt_attn_shape* shape, int s_h, int s
   p.out_T = shape->T;
   p.out_group = g.N;
   p.out = static_cast<uint16_t*>(out);
+  p.out_elems = static_cast<long long>(g.N) * g.H * 64;
   p.status = L.w.status;
   p.timeout_ns = kDefaultTimeoutNs;
   const int n_d = g.N - g.Nk;
@@ -991,6 +997,7 @@ extern "C" int vggt_attn_global_desc(const vggt_attn_shape* shape, int s_h, int 
   p.out_T = shape->T;
   p.out_group = g.N;
   p.out = static_cast<uint16_t*>(out);
+  p.out_elems = static_cast<long long>(g.N) * g.H * 64;
   p.status = L.w.status;
   p.timeout_ns = kDefaultTimeoutNs;
   ModeGeometry mg{1, g.N, g.N, 2};
@@ -1440,6 +1447,7 @@ extern "C" int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int wor
   p.out_T = shape->T;
   p.out_group = static_cast<int>(L.L);
   p.out = static_cast<uint16_t*>(out);
+  p.out_elems = static_cast<long long>(shape->S) * shape->T * shape->H * 64;
   p.status = L.w.status;
   p.timeout_ns = kDefaultTimeoutNs;
   ModeGeometry g{1, L.L, L.L, 2};
@@ -1604,6 +1612,7 @@ extern "C" int vggt_attn_global_shard_core_peers(const vggt_attn_shape* shape, i
   p.out_T = shape->T;
   p.out_group = static_cast<int>(L.L);
   p.out = static_cast<uint16_t*>(out);
+  p.out_elems = static_cast<long long>(shape->S) * shape->T * shape->H * 64;
   p.status = L.w.status;
   p.timeout_ns = kDefaultTimeoutNs;
   p.rank_tokens = static_cast<int>(L.L);
