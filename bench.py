@@ -806,6 +806,9 @@ def run_one(args) -> int:
     shape = W.workload(args.workload).shape
     if args.frames > 0:
         shape = dataclasses.replace(shape, S=args.frames)
+    if args.patch_grid is not None:   # e.g. 0 0: frames of special tokens only (register mode's whole input)
+        gh, gw = args.patch_grid
+        shape = dataclasses.replace(shape, grid_h=gh, grid_w=gw, T=shape.n_special + gh * gw)
     g = torch.Generator(device="cuda")
     g.manual_seed(1234)
     H, C = shape.H, shape.H * 64
@@ -862,6 +865,9 @@ def main():
                          "exit: a small case for ncu")
     ap.add_argument("--frames", type=int, default=0, help="with --one: override the frame count S")
     ap.add_argument("--calls", type=int, default=3, help="with --one: timed calls after one warm-up call")
+    ap.add_argument("--patch-grid", type=int, nargs=2, default=None, metavar=("H", "W"),
+                    help="with --one: override the patch grid (0 0: special tokens only, a small input that gives "
+                         "register mode its full problem)")
     ap.add_argument("--block", action="store_true", help="with --one: a whole transformer block")
     ap.add_argument("--sga", type=int, default=0, help="with --one global: subsampled global attention, s x s grid")
     ap.add_argument("--desc", type=int, default=0, help="with --one global: descriptor attention, s x s windows")
