@@ -76,6 +76,15 @@ def shard_plan(world: int, rank: int, base_seed: int):
     return {"rank": rank, "world": world, "seed": base_seed + 7919 * rank, "problems": 1}
 
 
+def scene_frames(S: int, world: int, rank: int) -> range:
+    """Query-sharded global attention: rank r holds frames [r * S / world, (r + 1) * S / world) of the scene
+    (consecutive blocks in rank order, the order the all-gather concatenates the ranks' keys in)."""
+    if S % world:
+        raise ValueError(f"--sharded splits the {S} frames evenly: {world} ranks do not divide them")
+    per = S // world
+    return range(rank * per, (rank + 1) * per)
+
+
 def reduce_max(value: float, device=None) -> float:
     """Max of a scalar over all ranks (identity without a process group)."""
     import torch
@@ -442,6 +451,109 @@ def run_ours(args):
             "e2e": e2e, "roofline": roofline, "gpu_launches": launches, "clocks": clk, "cpu_baseline": cpu}
     if side:   # side measurements (blocks, subsampled and sharded forms) on a line of their own, before the result
         print(json.dumps({"side_measurements": side}), flush=True)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_sharded(args):
+    """--sharded: one scene (the 100-frame global workload) split across the ranks by frames; every step is
+    query-sharded global attention (vit_attention_b200.sharded.global_attention_sharded: the rank's prologue,
+    one NCCL all-gather each of the normalised keys and of the values, the rank's core over all keys).
+    `value` = the scene's algorithmic flops per step / the max-over-ranks time ("scaling": "strong"); `e2e`
+    adds, every step, the H2D of the rank's qkv frames from pinned host memory and the D2H of its output
+    rows (serialised with the step on the rank's stream)."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    import vit_attention_b200 as V
+    from vit_attention_b200.sharded import global_attention_sharded
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(device)
+    stream = torch.cuda.current_stream(device)
+    w = W.workload(HEADLINE)
+    frames = scene_frames(w.shape.S, world, rank)
+    shape = dataclasses.replace(w.shape, S=len(frames))
+    x = W.make_qkv(w.shape, w.seed, w.lowrank, frames)
+    prm = W.make_norm_params(w.shape.H, w.seed)
+    qkv = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+    g = {k: torch.from_numpy(np.ascontiguousarray(prm[k])).to(device) for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}
+    out = torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(V.vggt_attn_shard_workspace_size(shape, world), dtype=torch.uint8, device=device)
+
+    def step():
+        global_attention_sharded(shape, qkv, g["q_gamma"], g["q_beta"], g["k_gamma"], g["k_beta"], out, ws,
+                                 stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    assert V.vggt_attn_read_status(ws, stream) == 0
+    clocks = ClockSampler(device.index)
+    clocks.start()
+    time.sleep(0.4)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for _ in range(args.steps):
+        step()
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    clk = clocks.stop()
+    ms = reduce_max(t0.elapsed_time(t1), device)
+    assert V.vggt_attn_read_status(ws, stream) == 0
+    flops = attention_flops("global", w.shape)                 # the whole scene's work per step
+    value = flops * args.steps / (ms / 1000.0) / 1e12
+    # e2e: the rank's frames in from pinned host memory and its output rows back, every step
+    h_qkv = torch.empty(qkv.shape, dtype=torch.bfloat16, pin_memory=True)
+    h_qkv.copy_(qkv)
+    h_out = torch.empty(out.shape, dtype=torch.bfloat16, pin_memory=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        qkv.copy_(h_qkv, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    # the scene's per-rank core alone (the all-gather and the prologue excluded), for the roofline
+    k_send, v_send, k_all, v_all = V.vggt_attn_shard_buffers(shape, world, ws)
+    core_ms = reduce_max(cuda_time_ms(lambda: V.vggt_attn_global_shard_core(shape, world, out, ws, None, stream),
+                                      stream, max(3, args.steps)), device)
+    peaks, peak_src = load_peaks()
+    peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    core_tflops = flops / world / (core_ms / 1000.0) / 1e12
+    gather_bytes = 2 * (world - 1) * k_send.numel() * 2
+    if world > 1:
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    cfg = headline_config(w, world)
+    cfg["parallelism"] = f"query-sharded x{world} over frames, NCCL all-gather of k and v (strong)"
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
+            "e2e": {"value": flops * args.steps / (e2e_ms / 1000.0) / 1e12, "unit": UNIT,
+                    "h2d_bytes_per_step": qkv.numel() * 2, "d2h_bytes_per_step": out.numel() * 2,
+                    "ms_per_step": e2e_ms / args.steps, "per_rank_bytes": True},
+            "roofline": {"bound": "tensor", "achieved": core_tflops, "peak": peak, "unit": "TFLOP/s",
+                         "frac": core_tflops / peak, "traffic": None,
+                         "kernel": "vggt::attn_core_kernel<CoreCfg<2, false, true>> (one rank's queries, all keys)",
+                         "kernel_ms": core_ms, "peak_source": f"{peak_src} bf16_tflops_sustained",
+                         "allgather_bytes_per_rank": gather_bytes},
+            "gpu_launches": 2 * args.steps, "clocks": clk, "cpu_baseline": None}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -860,6 +972,9 @@ def main():
     ap.add_argument("--linear-only", default=None, metavar="M,N,K",
                     help="run vggt_linear on an M x N x K problem a few times and exit (a small case for ncu)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sharded", action="store_true",
+                    help="one 100-frame scene split across the ranks by frames: query-sharded global attention with "
+                         "an NCCL all-gather of the keys and values (strong scaling; the ranks must divide 100)")
     ap.add_argument("--one", choices=("frame", "global", "register"), default=None,
                     help="run only this mode on --workload's shape (--frames, --calls, --block, --sga, --desc) and "
                          "exit: a small case for ncu")
@@ -880,6 +995,8 @@ def main():
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.sharded:
+        return run_sharded(args)
     return run_ours(args)
 
 

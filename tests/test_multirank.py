@@ -92,3 +92,68 @@ def test_sharded_global_gathers_kv_in_rank_order():
         k, v = res[r]
         assert k == [1.0] * 5 + [2.0] * 5
         assert v == [-1.5] * 5 + [-2.5] * 5
+
+
+# ---------------------------------------------------------------- bench --sharded: one scene split by frames
+def test_scene_frames_partition_covers_the_scene_in_rank_order():
+    import bench
+    for world in (1, 2, 4, 5):
+        parts = [bench.scene_frames(100, world, r) for r in range(world)]
+        assert [f for p in parts for f in p] == list(range(100))
+        assert len({len(p) for p in parts}) == 1
+    with pytest.raises(ValueError):
+        bench.scene_frames(100, 8, 0)
+
+
+def test_frame_range_draw_equals_the_whole_scene_draw():
+    import numpy as np
+    import workloads as W
+    shape = W.Shape(S=6, T=9, H=2, n_special=1, grid_h=2, grid_w=4)
+    full = W.make_qkv(shape, 1234, 0.5)
+    np.testing.assert_array_equal(W.make_qkv(shape, 1234, 0.5, range(2, 5)), full[2:5])
+    np.testing.assert_array_equal(W.make_qkv(shape, 1234, 0.0, range(0, 6)), W.make_qkv(shape, 1234, 0.0))
+
+
+def _scene_worker(rank, world, port, results):
+    import datetime
+    import sys
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    sys.path.insert(0, root)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    import bench
+    import workloads as W
+    from vit_attention_b200.sharded import gather_kv
+    shape = W.Shape(S=4, T=5, H=2, n_special=1, grid_h=2, grid_w=2)
+    frames = bench.scene_frames(shape.S, world, rank)
+    mine = W.make_qkv(shape, 77, 0.5, frames)                       # [S/world, T, 3, H, 64] bits
+    # this rank's keys and values token-major, as the shard prologue's send buffers hold them
+    k_send = torch.from_numpy(mine[:, :, 1].reshape(-1, shape.H, 64).astype(np.float32))
+    v_send = torch.from_numpy(mine[:, :, 2].reshape(-1, shape.H, 64).astype(np.float32))
+    k_all = torch.empty((world * k_send.shape[0], shape.H, 64))
+    v_all = torch.empty_like(k_all)
+    gather_kv(k_send, v_send, k_all, v_all)
+    full = W.make_qkv(shape, 77, 0.5)
+    ok_k = np.array_equal(k_all.numpy(), full[:, :, 1].reshape(-1, shape.H, 64).astype(np.float32))
+    ok_v = np.array_equal(v_all.numpy(), full[:, :, 2].reshape(-1, shape.H, 64).astype(np.float32))
+    results[rank] = (list(frames), ok_k, ok_v, bench.reduce_max(float(rank)))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_sharded_scene_gathers_the_whole_scene_on_every_rank():
+    """bench --sharded's host side on 2 gloo ranks: each rank draws only its frames, and the all-gather in rank
+    order rebuilds the whole scene's keys and values exactly (the layout the shard core reads)."""
+    world = 2
+    port = _free_port()
+    with mp.get_context("spawn").Manager() as m:
+        results = m.dict()
+        mp.spawn(_scene_worker, args=(world, port, results), nprocs=world, join=True)
+        res = dict(results)
+    assert res[0][0] == [0, 1] and res[1][0] == [2, 3]
+    for r in range(world):
+        assert res[r][1] and res[r][2]
+        assert res[r][3] == 1.0

@@ -121,32 +121,35 @@ def make_norm_params(H: int, seed: int, head_dim: int = HEAD_DIM) -> Dict[str, n
     return out
 
 
-def make_qkv(shape: Shape, seed: int, lowrank: float = 0.0) -> np.ndarray:
+def make_qkv(shape: Shape, seed: int, lowrank: float = 0.0, frames: Optional[range] = None) -> np.ndarray:
     """Seeded bf16 ``qkv[S, T, 3, H, head_dim]`` bit patterns (uint16).
 
     Frame ``s`` is drawn from its own generator ``default_rng([seed, 0, s])``,
     so frames can be drawn in parallel and the result does not depend on the
-    number of threads.
+    number of threads.  ``frames`` (a range of frame indices) draws only those
+    frames, ``[len(frames), T, 3, H, head_dim]``, equal to the same frames of
+    the whole draw (a rank's share of a scene split by frames).
     """
     S, T, H, D = shape.S, shape.T, shape.H, shape.head_dim
+    frames = range(S) if frames is None else frames
     shared = None
     if lowrank:
         shared = (lowrank * np.random.default_rng([seed, 3]).standard_normal(
             (T, 3, H, D), dtype=np.float32)).astype(np.float32)
-    bits = np.empty((S, T, 3, H, D), dtype=np.uint16)
+    bits = np.empty((len(frames), T, 3, H, D), dtype=np.uint16)
 
-    def draw(s: int) -> None:
-        z = np.random.default_rng([seed, 0, s]).standard_normal((T, 3, H, D), dtype=np.float32)
+    def draw(i: int) -> None:
+        z = np.random.default_rng([seed, 0, frames[i]]).standard_normal((T, 3, H, D), dtype=np.float32)
         if shared is not None:
             z += shared
-        bits[s] = f32_to_bf16_bits(z)
+        bits[i] = f32_to_bf16_bits(z)
 
-    if S * T * 3 * H * D >= (1 << 22):
+    if len(frames) * T * 3 * H * D >= (1 << 22):
         with concurrent.futures.ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as ex:
-            list(ex.map(draw, range(S)))
+            list(ex.map(draw, range(len(frames))))
     else:
-        for s in range(S):
-            draw(s)
+        for i in range(len(frames)):
+            draw(i)
     return bits
 
 
