@@ -22,7 +22,12 @@
 // against 8 per 64, the per-instruction cost of these small products being
 // what paces the loop), and row sums kept in registers by the softmax threads
 // (fp32 sums of the probabilities before their rounding to bf16) instead of
-// 16 ones columns in the PV product.  Barrier phases run on across units.
+// 16 ones columns in the PV product.  From its second step on, a tile's
+// exponentials run against the reference max as it stands while the step's
+// row max is taken in the same loop (ALU work beside the MUFU work, instead of
+// a max pass ahead of them); in the rare step whose max exceeds the reference
+// by more than the threshold they are redone against the new max, so P is the
+// same as with the max taken first.  Barrier phases run on across units.
 // Every wait is bounded.
 #pragma once
 
@@ -185,25 +190,31 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
         for (int e = 0; e < BN; ++e)
           if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
       }
-      float mx0 = -INFINITY, mx1 = -INFINITY;
+      // Reference max for this step's exponentials: the running one, or on a
+      // tile's first step this step's own max (taken first).
+      float m_use = m_run;
+      if (j == 0) {
+        float a0 = -INFINITY, a1 = -INFINITY;
 #pragma unroll
-      for (int e = 0; e < BN; e += 4) {
-        mx0 = max3f(mx0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
-        mx1 = max3f(mx1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+        for (int e = 0; e < BN; e += 4) {
+          a0 = max3f(a0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+          a1 = max3f(a1, __uint_as_float(sr[e + 2]), __uint_as_float(sr[e + 3]));
+        }
+        m_use = fmaxf(a0, a1);
+        m_run = m_use;
       }
-      const float tile_max = fmaxf(mx0, mx1);
-      const bool move = (j == 0) || (tile_max > m_run + core::RESCALE_THRESHOLD);
-      float alpha = 1.f;
-      if (move) {
-        alpha = (j == 0) ? 0.f : ex2_approx(m_run - tile_max);
-        m_run = tile_max;
-      }
-      const float neg_m = -m_run;
-      {
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+      float l0 = 0.f, l1 = 0.f;
+      auto exps = [&](float neg_m, bool track) {
         uint32_t pk[BN / 2];
-        float l0 = 0.f, l1 = 0.f;
+        l0 = 0.f;
+        l1 = 0.f;
 #pragma unroll
         for (int e = 0; e < BN; e += 2) {
+          if (track) {
+            if ((e & 2) == 0) mx0 = max3f(mx0, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+            else mx1 = max3f(mx1, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]));
+          }
           float x0, x1, p0, p1;
           add_x2(__uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), neg_m, neg_m, x0, x1);
           const int pair = e >> 1;
@@ -216,13 +227,25 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
           add_x2(l0, l1, p0, p1, l0, l1);
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        // Row sum: this step's fp32 probabilities (two add chains) on top of
-        // the running sum, which moves with the reference max as O does.
-        l_run = l_run * alpha + (l0 + l1);
         // P (80 keys -> 40 bf16-pair columns) overwrites the first 40 columns of this S buffer.
         tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(pk));
         tmem_st8(s_addr + 32, pk + 32);
+      };
+      exps(-m_use, true);
+      const float tile_max = fmaxf(mx0, mx1);
+      const bool move = (j > 0) && (tile_max > m_run + core::RESCALE_THRESHOLD);
+      float alpha = 1.f;
+      if (move) {
+        alpha = ex2_approx(m_run - tile_max);
+        m_run = tile_max;
       }
+      if (__any_sync(0xffffffffu, move)) {   // rare: P and its sum again against the moved max (warp-collective stores)
+        tmem_wait_st();
+        exps(-m_run, false);
+      }
+      // Row sum: this step's fp32 probabilities (two add chains) on top of
+      // the running sum, which moves with the reference max as O does.
+      l_run = l_run * alpha + (l0 + l1);
       // Rescale O after PV(j-1) (S(j+1) was issued after it; past the unit's
       // last S, the unit's first PV_DONE commit says so).
       if (__any_sync(0xffffffffu, move && j > 0)) {
