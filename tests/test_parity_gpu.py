@@ -113,6 +113,85 @@ def test_zero_variance_rows_and_uniform_attention():
     assert np.abs(got - want[None]).max() <= 2e-2
 
 
+def _directional_inputs(shape, seed, angle_of_key):
+    """Special tokens only (no rotation); per head q = u and k = cos(a_t) u + sin(a_t) w (u, w zero-mean,
+    orthogonal, of equal norm, so LayerNorm keeps the angle) plus small noise, with gamma 2.5 so that the
+    scores, 72 cos(a_t) in base 2, span about +-72: keys whose angle shrinks along the sequence move the
+    running reference max by far more than its threshold after the first key step."""
+    import numpy as np
+    x = W.make_random_inputs(shape, seed)
+    rng = np.random.default_rng(seed)
+    u = rng.standard_normal((shape.H, 64))
+    u -= u.mean(-1, keepdims=True)
+    w = rng.standard_normal((shape.H, 64))
+    w -= w.mean(-1, keepdims=True)
+    w -= (w * u).sum(-1, keepdims=True) / (u * u).sum(-1, keepdims=True) * u
+    w *= np.linalg.norm(u, axis=-1, keepdims=True) / np.linalg.norm(w, axis=-1, keepdims=True)
+    a = np.array([angle_of_key(t) for t in range(shape.T)])
+    kdir = np.cos(a)[:, None, None] * u[None] + np.sin(a)[:, None, None] * w[None]        # [T, H, 64]
+    noise = lambda: 0.02 * rng.standard_normal((shape.S, shape.T, shape.H, 64))
+    x["qkv"][:, :, 0] = W.f32_to_bf16_bits((u[None, None] + noise()).astype(np.float32))
+    x["qkv"][:, :, 1] = W.f32_to_bf16_bits((kdir[None] + noise()).astype(np.float32))
+    for k in ("q_gamma", "k_gamma"):
+        x[k][:] = 2.5
+    for k in ("q_beta", "k_beta"):
+        x[k][:] = 0.0
+    return x
+
+
+LATE_MAX = [
+    ("step", lambda T: (lambda t: np.pi if t < 120 else 0.0)),      # one jump inside the second key step
+    ("ramp", lambda T: (lambda t: np.pi * (1.0 - t / (T - 1)))),    # the max grows at every step
+]
+
+
+def _bf16_storage_rows(mode, shape, x, queries):
+    """The attention of ``queries`` with the path's bf16 storage points applied to the fp64 computation
+    (shapes without patch tokens, so no rotation): q-hat (LayerNorm, gamma/beta, times softmax_scale *
+    log2(e)) and k-hat rounded to bf16, probabilities 2^(s - row max) rounded to bf16 for the product with v,
+    their sum unrounded.  Frame mode attends within the query's frame, global and register mode over all
+    tokens (every token is special here)."""
+    from block_tolerance import bf16_round
+    qkv = O.bf16_to_f64(x["qkv"])                                   # [S, T, 3, H, 64]
+    def ln(v, g, b):
+        m = v.mean(-1, keepdims=True)
+        return (v - m) / np.sqrt(((v - m) ** 2).mean(-1, keepdims=True) + shape.ln_eps) * g + b
+    scale = 0.125 * np.log2(np.e)
+    q = bf16_round(ln(qkv[:, :, 0], x["q_gamma"], x["q_beta"]) * scale)
+    k = bf16_round(ln(qkv[:, :, 1], x["k_gamma"], x["k_beta"]))
+    v = qkv[:, :, 2]
+    out = np.empty((len(queries), shape.H, 64))
+    for n, i in enumerate(queries):
+        f, t = divmod(int(i), shape.T)
+        kk, vv = (k[f], v[f]) if mode == "frame" else (k.reshape(-1, shape.H, 64), v.reshape(-1, shape.H, 64))
+        sc = np.einsum("hd,khd->hk", q[f, t], kk)
+        p = np.exp2(sc - sc.max(1, keepdims=True))
+        out[n] = np.einsum("hk,khd->hd", bf16_round(p), vv) / p.sum(1)[:, None]
+    return out
+
+
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
+@pytest.mark.parametrize("kind,angle", LATE_MAX, ids=[k for k, _ in LATE_MAX])
+def test_late_keys_move_the_reference_max(mode, kind, angle):
+    """The online softmax's reference max moves (by tens of units, base 2) after the first key step; in
+    frame mode the step's exponentials are then redone against the moved max.  Every query row is compared
+    with the oracle.  Scores of +-72 magnify the bf16 rounding of q-hat and k-hat (a score's error grows with
+    its size), so the bound is three times the error of the bf16 storage points alone on these inputs
+    (about 2e-2 relative, against 5e-3 for the workloads); a wrong rescale would be off by O(1)."""
+    from parity import errors
+    shape = W.Shape(S=3, T=400, H=2, n_special=400, grid_h=0, grid_w=1)
+    x = _directional_inputs(shape, 77, angle(shape.T))
+    out = run_gpu(mode, shape, x)
+    q = np.arange(shape.S * shape.T)
+    want = O.attn_mode(mode, shape, x, q)
+    got = rows(out, shape, q)
+    assert np.all(np.isfinite(got))
+    e_max, e_rel = errors(got, want)
+    s_max, s_rel = errors(_bf16_storage_rows(mode, shape, x, q), want)
+    assert e_max <= 3 * s_max and e_rel <= 3 * s_rel, (kind, mode, e_max, e_rel, s_max, s_rel)
+    assert e_rel <= 0.05
+
+
 # ------------------------------------------------------------------ the workloads at full size (sampled)
 @pytest.mark.slow
 def test_workload1_frame_full():
