@@ -93,6 +93,40 @@ def test_block_ragged_matches_oracle(mode):
     _block_case(mode, W.Shape(S=3, T=1031, H=16, n_special=17, grid_h=26, grid_w=39), 32, 512)
 
 
+@pytest.mark.parametrize("mode", ["frame", "global"])
+def test_block_wide_patch_grid_matches_oracle(mode):
+    # grid 2 x 420: 422 RoPE positions, more than the normalising GEMM epilogue keeps in shared memory beside
+    # its buffers, so the block takes the GEMM followed by the separate prologue instead.
+    _block_case(mode, W.Shape(S=2, T=845, H=4, n_special=5, grid_h=2, grid_w=420), 33, 256)
+
+
+def test_qkv_proj_matches_oracle_attention():
+    """vggt_attn_qkv_proj (the QKV GEMM whose epilogue normalises and rotates q and k into the workspace and
+    writes v into qkv) followed by vggt_attn_core: the attention output against the oracle on the projected
+    qkv."""
+    import torch
+    import vit_attention_b200 as V
+    for mode, shape in (("frame", W.Shape(S=3, T=1031, H=16, n_special=17, grid_h=26, grid_w=39)),
+                        ("global", W.workload(0).shape)):
+        blk = W.make_block_inputs(shape, 34)
+        C, M = shape.H * 64, shape.S * shape.T
+        dev = {k: _dev_bits(blk[k]) for k in ("x", "w_qkv")}
+        dev.update({k: _dev_f32(blk[k]) for k in ("b_qkv", "q_gamma", "q_beta", "k_gamma", "k_beta")})
+        ws = torch.empty(V.vggt_attn_workspace_size(shape, mode), dtype=torch.uint8, device="cuda")
+        qkv = torch.empty((shape.S, shape.T, 3, shape.H, 64), dtype=torch.bfloat16, device="cuda")
+        attn = torch.empty((shape.S, shape.T, shape.H, 64), dtype=torch.bfloat16, device="cuda")
+        V.vggt_attn_qkv_proj(mode, shape, dev["x"], dev["w_qkv"], dev["b_qkv"], dev["q_gamma"], dev["q_beta"],
+                             dev["k_gamma"], dev["k_beta"], qkv, ws)
+        V.vggt_attn_core(mode, shape, qkv, attn, ws)
+        assert V.vggt_attn_read_status(ws) == 0
+        q = query_sample(mode, shape, 512, 35)
+        inputs = {"qkv_f64": O.projected_qkv(shape, blk)}
+        inputs.update({k: blk[k] for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")})
+        want = O.attn_mode(mode, shape, inputs, q)
+        got = attn.view(M, shape.H, 64).index_select(0, torch.as_tensor(q, device="cuda")).float().cpu().numpy()
+        assert_close(got.astype(np.float64), want, f"qkv_proj + core {mode}")
+
+
 def test_qkv_proj_rejects_register_mode_and_odd_heads():
     import torch
     import vit_attention_b200 as V

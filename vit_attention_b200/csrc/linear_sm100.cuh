@@ -11,7 +11,7 @@
 //   resid  -- y = r + ls * Y with r a bf16 [M][N] residual and ls a per-column
 //             LayerScale vector, into y (may be r itself: each element is read
 //             by the thread that then writes it, before the chunk's store);
-//   qkv    -- the QKV projection of a frame or global attention block: the
+//   qkv    -- (EPI_QKV) the QKV projection of a frame or global attention block: the
 //             columns of a 64-wide head slice of q or k go through the QK
 //             LayerNorm, the 2D RoPE and (q) the softmax scale in fp32 straight
 //             from the accumulator and land in the attention workspace in the
@@ -33,11 +33,13 @@
 //                (qkv epilogue: normalises and rotates), and writes its 128-byte
 //                row of the chunk into the staging buffer; one thread stores
 //                the chunk with TMA.
-//   warps 8-11   (gelu and resid epilogues only, 384 threads) a second
+//   warps 8-11   (gelu, resid and qkv epilogues, 384 threads) a second
 //                epilogue warpgroup: warps 4-7 take chunks 0-1 of every tile,
 //                warps 8-11 chunks 2-3, each with its own staging buffer, so
 //                that the heavier per-element work keeps up with the products
-//                (5 % off a frame-mode transformer block).
+//                (5 % off a frame-mode transformer block for gelu/resid).  The
+//                qkv epilogue also keeps its cos/sin table in shared memory, so
+//                its operand ring has 3 stages instead of 4 to make room.
 // Every mbarrier wait is bounded (wait_bounded); on expiry the CTA records
 // VGGT_ATTN_ERR_TIMEOUT in the status word and drains what it has in flight.
 #pragma once
@@ -50,13 +52,16 @@ namespace vggt {
 
 namespace lin {
 constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-enum { EPI_STD = 0, EPI_GELU = 1, EPI_RESID = 2 };     // EPI_STD: plain or qkv (LinearParams::fused)
+enum { EPI_STD = 0, EPI_GELU = 1, EPI_RESID = 2, EPI_QKV = 3 };
 constexpr int A_BYTES = BM * BK * 2;                   // 16 KB
 constexpr int B_BYTES = BN * BK * 2;                   // 32 KB
+// Operand ring stages: 4, or 3 for the qkv epilogue (its cos/sin table and a
+// second staging buffer take the fourth stage's shared memory).
+__host__ __device__ constexpr int stages_for(int epi) { return epi == EPI_QKV ? 3 : STAGES; }
 constexpr int OFF_A = 0;
-constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
-constexpr int OFF_STAGE = OFF_B + STAGES * B_BYTES;    // 128 x 64 bf16 output chunk (16 KB)
-constexpr int OFF_BAR = OFF_STAGE + BM * 128;
+__host__ __device__ constexpr int off_b(int epi) { return OFF_A + stages_for(epi) * A_BYTES; }
+__host__ __device__ constexpr int off_stage(int epi) { return off_b(epi) + stages_for(epi) * B_BYTES; }  // 128 x 64 bf16 chunk
+__host__ __device__ constexpr int off_bar(int epi) { return off_stage(epi) + BM * 128; }
 enum {
   BAR_FULL = 0,
   BAR_EMPTY = BAR_FULL + STAGES,
@@ -69,14 +74,15 @@ enum {
   BAR_DRAIN = BAR_STAGE_FREE2 + 1,
   N_BARS = BAR_DRAIN + 1
 };
-constexpr int OFF_MISC = OFF_BAR + N_BARS * 8;         // tmem slot, abort flag
-constexpr int OFF_ROPE = OFF_MISC + 16;                // cos/sin table (qkv epilogue)
+__host__ __device__ constexpr int off_misc(int epi) { return off_bar(epi) + N_BARS * 8; }   // tmem slot, abort flag
+__host__ __device__ constexpr int off_rope(int epi) { return off_misc(epi) + 16; }          // cos/sin table (qkv)
 constexpr int THREADS = 256;
-// The GELU and residual epilogues do more per element: they run on two
+// The GELU, residual and qkv epilogues do more per element: they run on two
 // warpgroups (warps 4-7 take the tile's first two 64-column chunks, warps
 // 8-11 the last two), each with its own staging buffer; the second buffer
-// sits where the qkv epilogue keeps its RoPE table.
-constexpr int OFF_STAGE2 = (OFF_ROPE + 1023) & ~1023;
+// follows the cos/sin table of (grid_h + grid_w) positions (none but qkv).
+__host__ __device__ constexpr int rope_bytes(int epi, int n_pos) { return epi == EPI_QKV ? n_pos * 16 * 8 : 0; }
+__host__ __device__ constexpr int off_stage2(int epi, int n_pos) { return (off_rope(epi) + rope_bytes(epi, n_pos) + 1023) & ~1023; }
 __host__ __device__ constexpr int epi_warpgroups(int epi) { return epi == EPI_STD ? 1 : 2; }
 __host__ __device__ constexpr int threads_for(int epi) { return 128 * (1 + epi_warpgroups(epi)); }
 constexpr uint32_t TMEM_COLS = 512;                    // two 256-column accumulators
@@ -102,9 +108,10 @@ struct LinearParams {
   const float* ls;             // [N]
 };
 
+// + 1 KB of slack to align the base to 1024 B
 __host__ __device__ constexpr int linear_smem_bytes(int grid_h, int grid_w, int epi = lin::EPI_STD) {
-  if (epi != lin::EPI_STD) return lin::OFF_STAGE2 + lin::BM * 128 + 1024;
-  return lin::OFF_ROPE + (grid_h + grid_w) * 16 * 8 + 1024;   // + slack to align the base to 1024 B
+  if (epi != lin::EPI_STD) return lin::off_stage2(epi, grid_h + grid_w) + lin::BM * 128 + 1024;
+  return lin::off_rope(epi) + 1024;
 }
 
 // 32 lanes x 64 columns load.
@@ -199,8 +206,8 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
         }
       }
     }
-    const int c = (EPI == lin::EPI_STD && p.fused) ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
-    const int h = (EPI == lin::EPI_STD && p.fused) ? (col0 / 64) % p.H : 0;   // plain GEMMs have H = 0
+    const int c = EPI == lin::EPI_QKV ? col0 / (p.H * 64) : 2;   // 0 q, 1 k, 2 v (or plain)
+    const int h = EPI == lin::EPI_QKV ? (col0 / 64) % p.H : 0;
     uint4 o[8];
     if (c == 2) {
 #pragma unroll
@@ -210,7 +217,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
         o[k].z = pack_bf16x2(__uint_as_float(v[8 * k + 4]), __uint_as_float(v[8 * k + 5]));
         o[k].w = pack_bf16x2(__uint_as_float(v[8 * k + 6]), __uint_as_float(v[8 * k + 7]));
       }
-    } else if constexpr (EPI == lin::EPI_STD) {
+    } else if constexpr (EPI == lin::EPI_QKV) {
       // QK LayerNorm over the head's 64 values (biased variance, two passes;
       // eight partial sums each, then a short tree).
       float ps[8];
@@ -245,7 +252,9 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
         const float2* cs = rope_tab + (hf == 0 ? prow : p.grid_h + pcol) * 16;
-        float y[32];
+        // Dims d0..d0+3 and their RoPE partners d1 = d0 + 16: packed straight
+        // into the output words (o[4 hf + j/8] holds dims 32 hf + j/8*8 ..,
+        // o[4 hf + 2 + j/8] the partners).
 #pragma unroll
         for (int j = 0; j < 16; j += 4) {
           const int d0 = 32 * hf + j, d1 = d0 + 16;
@@ -255,6 +264,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
           const float4 b1 = __ldg(reinterpret_cast<const float4*>(bt + d1));
           const float ga[4] = {g0.x, g0.y, g0.z, g0.w}, gb[4] = {g1.x, g1.y, g1.z, g1.w};
           const float ba[4] = {b0.x, b0.y, b0.z, b0.w}, bb[4] = {b1.x, b1.y, b1.z, b1.w};
+          float ya[4], yb[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
             float a = __uint_as_float(v[d0 + i]) * rstd * ga[i] + ba[i];
@@ -265,16 +275,22 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
               bv = bv * w.x + a * w.y;
               a = a2;
             }
-            y[j + i] = a * mult;
-            y[j + i + 16] = bv * mult;
+            ya[i] = a * mult;
+            yb[i] = bv * mult;
           }
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          o[4 * hf + k].x = pack_bf16x2(y[8 * k], y[8 * k + 1]);
-          o[4 * hf + k].y = pack_bf16x2(y[8 * k + 2], y[8 * k + 3]);
-          o[4 * hf + k].z = pack_bf16x2(y[8 * k + 4], y[8 * k + 5]);
-          o[4 * hf + k].w = pack_bf16x2(y[8 * k + 6], y[8 * k + 7]);
+          uint4& oa = o[4 * hf + j / 8];
+          uint4& ob = o[4 * hf + 2 + j / 8];
+          if ((j & 4) == 0) {
+            oa.x = pack_bf16x2(ya[0], ya[1]);
+            oa.y = pack_bf16x2(ya[2], ya[3]);
+            ob.x = pack_bf16x2(yb[0], yb[1]);
+            ob.y = pack_bf16x2(yb[2], yb[3]);
+          } else {
+            oa.z = pack_bf16x2(ya[0], ya[1]);
+            oa.w = pack_bf16x2(ya[2], ya[3]);
+            ob.z = pack_bf16x2(yb[0], yb[1]);
+            ob.w = pack_bf16x2(yb[2], yb[3]);
+          }
         }
       }
     }
@@ -297,7 +313,7 @@ __device__ __forceinline__ bool linear_epilogue(const LinearParams& p, uint32_t 
       ok = wait_bounded(bar(bar_full), chunk & 1, abort_flag, p.status, p.timeout_ns, 0x550u);
       if (ok) {
         const uint32_t src = smem_addr(stage);
-        if (EPI != lin::EPI_STD || !p.fused)
+        if (EPI != lin::EPI_QKV)
           tma_store_3d(to0, src, col0, m0, 0);          // y [M][N]
         else if (c == 2)
           tma_store_4d(to0, src, 0, h, 2, m0);          // v slot of qkv [M][3][H][64]
@@ -318,6 +334,8 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
                   const __grid_constant__ CUtensorMap tmap_o0, const __grid_constant__ CUtensorMap tmap_o1,
                   const __grid_constant__ CUtensorMap tmap_o2, const LinearParams p) {
   using namespace lin;
+  constexpr int NST = stages_for(EPI);
+  constexpr int OFF_B = off_b(EPI), OFF_STAGE = off_stage(EPI), OFF_BAR = off_bar(EPI), OFF_MISC = off_misc(EPI);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_addr(smem);
@@ -325,14 +343,14 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
   auto bar = [&](int i) { return bar0 + 8u * static_cast<uint32_t>(i); };
   volatile uint32_t* tmem_slot = reinterpret_cast<volatile uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
-  float2* rope_tab = reinterpret_cast<float2*>(smem + OFF_ROPE);
+  float2* rope_tab = reinterpret_cast<float2*>(smem + off_rope(EPI));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int tiles_m = (p.M + BM - 1) / BM, tiles_n = p.N / BN, n_tiles = tiles_m * tiles_n;
   const int k_steps = p.K / BK;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(bar(BAR_FULL + s), 1);
       mbar_init(bar(BAR_EMPTY + s), 1);
     }
@@ -354,12 +372,12 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
     tma_prefetch_desc(&tmap_x);
     tma_prefetch_desc(&tmap_w);
     tma_prefetch_desc(&tmap_o0);
-    if (p.fused) {
+    if (EPI == EPI_QKV) {
       tma_prefetch_desc(&tmap_o1);
       tma_prefetch_desc(&tmap_o2);
     }
   }
-  if (p.fused) {
+  if (EPI == EPI_QKV) {
     const int n_pos = p.grid_h + p.grid_w;
     for (int e = threadIdx.x; e < n_pos * 16; e += blockDim.x) {
       const int pos_idx = e >> 4, j = e & 15;
@@ -383,16 +401,16 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0 && !skip) {
-      int issued[STAGES];
-      for (int s = 0; s < STAGES; ++s) issued[s] = 0;
+      int issued[NST];
+      for (int s = 0; s < NST; ++s) issued[s] = 0;
       bool ok = true;
       int it = 0;
       for (int t = blockIdx.x; t < n_tiles && ok; t += gridDim.x) {
         const int m0 = (t / tiles_n) * BM, n0 = (t % tiles_n) * BN;
         for (int k = 0; k < k_steps; ++k, ++it) {
-          const int st = it % STAGES;
-          if (it >= STAGES) {
-            ok = wait_bounded(bar(BAR_EMPTY + st), ((it / STAGES) - 1) & 1, abort_flag, p.status, p.timeout_ns,
+          const int st = it % NST;
+          if (it >= NST) {
+            ok = wait_bounded(bar(BAR_EMPTY + st), ((it / NST) - 1) & 1, abort_flag, p.status, p.timeout_ns,
                               0x500u | st);
             if (!ok) break;
           }
@@ -403,7 +421,7 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
         }
       }
       if (!ok) {
-        for (int st = 0; st < STAGES; ++st)
+        for (int st = 0; st < NST; ++st)
           if (issued[st] > 0) wait_drain(bar(BAR_FULL + st), (issued[st] - 1) & 1, p.timeout_ns);
       }
     }
@@ -424,8 +442,8 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
         }
         const uint32_t d = tmem + ab * BN;
         for (int k = 0; k < k_steps; ++k, ++it) {
-          const int st = it % STAGES;
-          ok = wait_bounded(bar(BAR_FULL + st), (it / STAGES) & 1, abort_flag, p.status, p.timeout_ns, 0x520u | st);
+          const int st = it % NST;
+          ok = wait_bounded(bar(BAR_FULL + st), (it / NST) & 1, abort_flag, p.status, p.timeout_ns, 0x520u | st);
           if (!ok) break;
           tc_fence_after();
 #pragma unroll
@@ -449,7 +467,7 @@ __global__ void __launch_bounds__(lin::threads_for(EPI), 1)
       const int wg = (warp - 4) >> 2;                        // epilogue warpgroup
       constexpr int CPW = (BN / 64) / epi_warpgroups(EPI);   // chunks per warpgroup
       const bool leader = (threadIdx.x & 127) == 0;
-      uint8_t* stage = smem + (wg == 0 ? OFF_STAGE : OFF_STAGE2);
+      uint8_t* stage = smem + (wg == 0 ? OFF_STAGE : off_stage2(EPI, p.grid_h + p.grid_w));
       const uint32_t lane_base = static_cast<uint32_t>(quarter * 32) << 16;
       int lt = 0, chunk = 0;
       for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++lt) {

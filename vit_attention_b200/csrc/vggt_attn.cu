@@ -573,7 +573,6 @@ template <int EPI>
 int launch_linear_epi(const vggt::LinearParams& p, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& o0,
                       const CUtensorMap& o1, const CUtensorMap& o2, int smem, unsigned grid, cudaStream_t stream) {
   static_assert(vggt::linear_smem_bytes(0, 0, vggt::lin::EPI_GELU) <= 227 * 1024, "two staging buffers fit");
-  if (EPI != vggt::lin::EPI_STD) smem = vggt::linear_smem_bytes(0, 0, EPI);
   if (cudaFuncSetAttribute(vggt::linear_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return VGGT_ATTN_ERR_CUDA;
   vggt::linear_kernel<EPI><<<grid, vggt::lin::threads_for(EPI), smem, stream>>>(mx, mw, o0, o1, o2, p);
@@ -585,7 +584,7 @@ int launch_linear(vggt::LinearParams p, const void* x, const void* w, const CUte
   CUtensorMap mx, mw;
   if (!make_rows_map(&mx, x, p.K, p.M, vggt::lin::BM) || !make_rows_map(&mw, w, p.K, p.N, vggt::lin::BN))
     return VGGT_ATTN_ERR_CUDA;
-  const int smem = vggt::linear_smem_bytes(grid_h, grid_w);
+  const int smem = vggt::linear_smem_bytes(grid_h, grid_w, epi);
   if (smem > 227 * 1024) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -597,6 +596,7 @@ int launch_linear(vggt::LinearParams p, const void* x, const void* w, const CUte
   switch (epi) {
     case vggt::lin::EPI_GELU: return launch_linear_epi<vggt::lin::EPI_GELU>(p, mx, mw, o0, o1, o2, smem, grid, stream);
     case vggt::lin::EPI_RESID: return launch_linear_epi<vggt::lin::EPI_RESID>(p, mx, mw, o0, o1, o2, smem, grid, stream);
+    case vggt::lin::EPI_QKV: return launch_linear_epi<vggt::lin::EPI_QKV>(p, mx, mw, o0, o1, o2, smem, grid, stream);
     default: return launch_linear_epi<vggt::lin::EPI_STD>(p, mx, mw, o0, o1, o2, smem, grid, stream);
   }
 }
@@ -623,7 +623,7 @@ int check_qkv_proj_args(int mode, const vggt_attn_shape* s, const void* x, const
 
 int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
                     const float* gq, const float* bq, const float* gk, const float* bk, void* qkv,
-                    const WorkspaceView& wv, cudaStream_t stream) {
+                    const WorkspaceView& wv, cudaStream_t stream, bool zero_status = true) {
   const ModeGeometry g = geometry(s, mode);
   vggt::LinearParams p{};
   p.M = s->S * s->T;
@@ -631,7 +631,7 @@ int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const voi
   p.K = s->H * 64;
   p.bias = b;
   p.status = wv.status;
-  p.zero_status = 1;
+  p.zero_status = zero_status ? 1 : 0;
   p.fused = 1;
   p.gamma[0] = gq;
   p.gamma[1] = gk;
@@ -662,8 +662,19 @@ int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const voi
       return VGGT_ATTN_ERR_CUDA;
   }
   (void)g;
-  return launch_linear(p, x, w, mv, mq, mk, s->grid_h, s->grid_w, stream);
+  return launch_linear(p, x, w, mv, mq, mk, s->grid_h, s->grid_w, stream, vggt::lin::EPI_QKV);
 }
+
+// The QKV projection of an attention block with the QK-LayerNorm + RoPE:
+// the GEMM with the normalising epilogue (q and k straight into the
+// workspace planes, v into its slot of qkv; measured 4-8 % faster than the
+// plain GEMM followed by the prologue pass, which it replaces) when its
+// cos/sin table fits in shared memory beside the GEMM's buffers, else the
+// GEMM followed by the prologue.  zero_status: this is the call's first
+// kernel.
+int launch_block_qkv(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
+                     const float* gq, const float* bq, const float* gk, const float* bk, void* qkv,
+                     const WorkspaceView& wv, cudaStream_t stream, bool zero_status);
 
 }  // namespace
 
@@ -747,6 +758,17 @@ int launch_linear_plain(const void* x, const void* w, const float* b, void* y, l
   return launch_linear(p, x, w, my, my, my, 0, 0, st, epi);
 }
 
+int launch_block_qkv(int mode, const vggt_attn_shape* s, const void* x, const void* w, const float* b,
+                     const float* gq, const float* bq, const float* gk, const float* bk, void* qkv,
+                     const WorkspaceView& wv, cudaStream_t stream, bool zero_status) {
+  if (vggt::linear_smem_bytes(s->grid_h, s->grid_w, vggt::lin::EPI_QKV) <= 227 * 1024)
+    return launch_qkv_proj(mode, s, x, w, b, gq, bq, gk, bk, qkv, wv, stream, zero_status);
+  const long long M = static_cast<long long>(s->S) * s->T, C = static_cast<long long>(s->H) * 64;
+  int rc = launch_linear_plain(x, w, b, qkv, M, 3 * C, C, wv.status, stream, zero_status);
+  if (rc) return rc;
+  return launch_prologue(mode, s, qkv, gq, bq, gk, bk, wv, stream, false);
+}
+
 int check_block_args(int mode, const vggt_attn_shape* s, const void* x, const void* w_qkv, const float* b_qkv,
                      const float* gq, const float* bq, const float* gk, const float* bk, const void* w_out,
                      const float* b_out, void* qkv, void* attn, void* y, void* ws, size_t ws_bytes) {
@@ -797,19 +819,16 @@ extern "C" int vggt_attn_block(int mode, const vggt_attn_shape* shape, const voi
     uint8_t* ys = as + Ms * row;
     const WorkspaceView wv = workspace_view(&s2, VGGT_ATTN_GLOBAL, workspace);
     if ((rc = launch_special_rows(x, xs, static_cast<int>(Ms), row, shape->n_special, shape->T, true, st))) return rc;
-    if ((rc = launch_linear_plain(xs, w_qkv, b_qkv, qkv, Ms, 3 * C, C, wv.status, st, true))) return rc;
-    if ((rc = launch_prologue(VGGT_ATTN_GLOBAL, &s2, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st, false)))
+    if ((rc = launch_block_qkv(VGGT_ATTN_GLOBAL, &s2, xs, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, wv, st,
+                               true)))
       return rc;
     if ((rc = launch_core(VGGT_ATTN_GLOBAL, &s2, qkv, as, wv, st))) return rc;
     if ((rc = launch_linear_plain(as, w_out, b_out, ys, Ms, C, C, wv.status, st))) return rc;
     return launch_special_rows(ys, y, static_cast<int>(Ms), row, shape->n_special, shape->T, false, st);
   }
   const WorkspaceView wv = workspace_view(shape, mode, workspace);
-  // QKV projection as a plain GEMM into qkv, then the prologue: measured
-  // faster than the fused projection (whose LayerNorm/RoPE epilogue, not its
-  // products, sets its time) on both the frame and the global workloads.
-  if ((rc = launch_linear_plain(x, w_qkv, b_qkv, qkv, M, 3 * C, C, wv.status, st, true))) return rc;
-  if ((rc = launch_prologue(mode, shape, qkv, q_gamma, q_beta, k_gamma, k_beta, wv, st, false))) return rc;
+  if ((rc = launch_block_qkv(mode, shape, x, w_qkv, b_qkv, q_gamma, q_beta, k_gamma, k_beta, qkv, wv, st, true)))
+    return rc;
   if ((rc = launch_core(mode, shape, qkv, attn, wv, st))) return rc;
   return launch_linear_plain(attn, w_out, b_out, y, M, C, C, wv.status, st);
 }
@@ -1136,8 +1155,8 @@ int run_block(int mode, const vggt_attn_shape* shape, void* x, const vggt_block_
   uint8_t* att = L.big + static_cast<size_t>(M) * 3 * C * 2;
   if ((rc = launch_layernorm(xb, L.h, w->norm1_gamma, w->norm1_beta, M, C, eps, status, clear_status, st)))
     return rc;
-  if ((rc = launch_linear_plain(L.h, w->w_qkv, w->b_qkv, qkv, M, 3 * C, C, status, st))) return rc;
-  if ((rc = launch_prologue(L.mode, &L.s, qkv, w->q_gamma, w->q_beta, w->k_gamma, w->k_beta, L.att, st, false)))
+  if ((rc = launch_block_qkv(L.mode, &L.s, L.h, w->w_qkv, w->b_qkv, w->q_gamma, w->q_beta, w->k_gamma, w->k_beta, qkv,
+                              L.att, st, false)))
     return rc;
   if ((rc = launch_core(L.mode, &L.s, qkv, att, L.att, st))) return rc;
   if ((rc = launch_linear_plain(att, w->w_proj, w->b_proj, xb, M, C, C, status, st, false, vggt::lin::EPI_RESID, xb,
