@@ -241,7 +241,7 @@ __global__ void __launch_bounds__(PRO_MAX_THREADS) qk_norm_rope_kernel(const Pro
         ob.w = pack_bf16x2(xb[6] * mult, xb[7] * mult);
         const long long dst_off = (c == 1 && p.k_token_major) ? w[k].dst_v + h * 64 + base : w[k].dst_qk + row_dst;
         uint16_t* dst = p.ws_qk[c] + dst_off;
-        const long long dst_elems = (c == 1 && p.k_token_major) ? p.v_elems : p.qk_elems;
+        [[maybe_unused]] const long long dst_elems = (c == 1 && p.k_token_major) ? p.v_elems : p.qk_elems;
         if (VGGT_DBG_BOUNDS(dst_off + 24 <= dst_elems, p.status, 0x922u)) {
           *reinterpret_cast<uint4*>(dst) = oa;
           *reinterpret_cast<uint4*>(dst + 16) = ob;
