@@ -226,10 +226,11 @@ __device__ __forceinline__ void frame_softmax_role(const CoreParams& p, const Fr
           }
           add_x2(l0, l1, p0, p1, l0, l1);
           pk[e >> 1] = pack_bf16x2(p0, p1);
+          // P (80 keys -> 40 bf16-pair columns) over the first 40 columns of this S buffer, in parts as produced
+          if (e == 30) tmem_st16(s_addr, pk);
+          if (e == 62) tmem_st16(s_addr + 16, pk + 16);
+          if (e == 78) tmem_st8(s_addr + 32, pk + 32);
         }
-        // P (80 keys -> 40 bf16-pair columns) overwrites the first 40 columns of this S buffer.
-        tmem_st32(s_addr, *reinterpret_cast<const uint32_t(*)[32]>(pk));
-        tmem_st8(s_addr + 32, pk + 32);
       };
       exps(-m_use, true);
       const float tile_max = fmaxf(mx0, mx1);
