@@ -96,9 +96,8 @@ struct LinearParams {
   int* status;
   unsigned long long timeout_ns;
   int zero_status;            // clear the status word first (the first kernel of an attention block)
-  // qkv epilogue (fused == 1); N = 3 * H * 64, K = H * 64; the destinations
+  // qkv epilogue (EPI_QKV); N = 3 * H * 64, K = H * 64; the destinations
   // are the kernel's output tensor maps (v slot of qkv, q plane, k plane)
-  int fused;
   const float* gamma[2];
   const float* beta[2];
   int H, T, n_special, grid_h, grid_w;

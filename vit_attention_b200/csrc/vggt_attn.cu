@@ -568,7 +568,7 @@ int check_linear_dims(long long M, long long N, long long K) {
 }
 
 // Output maps: o0 = y [M][N] (plain) or the v slot of qkv [M][3][H][64]
-// (fused, as (64, H, 3, M)); o1, o2 = the q and k planes [H][M][64] (fused).
+// (qkv epilogue, as (64, H, 3, M)); o1, o2 = the q and k planes [H][M][64] (qkv epilogue).
 template <int EPI>
 int launch_linear_epi(const vggt::LinearParams& p, const CUtensorMap& mx, const CUtensorMap& mw, const CUtensorMap& o0,
                       const CUtensorMap& o1, const CUtensorMap& o2, int smem, unsigned grid, cudaStream_t stream) {
@@ -632,7 +632,6 @@ int launch_qkv_proj(int mode, const vggt_attn_shape* s, const void* x, const voi
   p.bias = b;
   p.status = wv.status;
   p.zero_status = zero_status ? 1 : 0;
-  p.fused = 1;
   p.gamma[0] = gq;
   p.gamma[1] = gk;
   p.beta[0] = bq;
