@@ -27,7 +27,9 @@
 // row max is taken in the same loop (ALU work beside the MUFU work, instead of
 // a max pass ahead of them); in the rare step whose max exceeds the reference
 // by more than the threshold they are redone against the new max, so P is the
-// same as with the max taken first.  Barrier phases run on across units.
+// same as with the max taken first.  P goes into TMEM in three stores issued
+// from inside the exponential loop as its parts are ready, so that the stores
+// overlap the remaining exponentials.  Barrier phases run on across units.
 // Every wait is bounded.
 #pragma once
 
