@@ -86,6 +86,26 @@ def test_mlp_branch_alone(mode, wts, x):
     np.testing.assert_allclose(O.block_forward(mode, SHAPE, x, w, EPS), want.numpy(), rtol=1e-11, atol=1e-11)
 
 
+@pytest.mark.parametrize("mode", ["frame", "global"])
+def test_full_block_runs_the_mlp_on_the_attention_branch_output(mode, wts, x):
+    """Both branches on: the MLP reads x + ls1 * attention branch (sequential
+    residuals, not two parallel branches on x), every step by torch."""
+    C = SHAPE.H * 64
+    xf = tw(x)
+    h = F.layer_norm(xf, (C,), t64(wts["norm1_gamma"]), t64(wts["norm1_beta"]), eps=EPS)
+    qkv = F.linear(h, tw(wts["w_qkv"]), t64(wts["b_qkv"])).numpy().reshape(SHAPE.S, SHAPE.T, 3, SHAPE.H, 64)
+    inputs = {"qkv_f64": qkv, **{k: wts[k] for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}}
+    a = t64(O.attn_mode(mode, SHAPE, inputs).reshape(-1, C))
+    xr = xf + t64(wts["ls1"]) * F.linear(a, tw(wts["w_proj"]), t64(wts["b_proj"]))
+    h2 = F.layer_norm(xr, (C,), t64(wts["norm2_gamma"]), t64(wts["norm2_beta"]), eps=EPS)
+    u = F.gelu(F.linear(h2, tw(wts["w_fc1"]), t64(wts["b_fc1"])), approximate="none")
+    want = xr + t64(wts["ls2"]) * F.linear(u, tw(wts["w_fc2"]), t64(wts["b_fc2"]))
+    got = O.block_forward(mode, SHAPE, x, wts, EPS)
+    np.testing.assert_allclose(got, want.numpy(), rtol=1e-11, atol=1e-11)
+    # the test has teeth: with the block's LayerScale the MLP branch changes the output measurably
+    assert np.abs(got - xr.numpy()).max() > 1e-8
+
+
 def test_register_block_changes_only_special_rows_like_a_global_block_on_them(wts, x):
     y = O.block_forward("register", SHAPE, x, wts, EPS)
     sp = O.register_tokens(SHAPE)

@@ -4,8 +4,9 @@ The attention block of the VGGT-Omega Aggregator explainer (section 3)
 projects token features to q, k, v and the attention output back; the oracle
 writes that out in fp64.  These tests pin it to things other than itself: a
 permutation weight (a transposed W would give the inverse permutation), torch's
-fp64 linear, and identity projections that reduce the block to the already
-pinned attention oracle.
+fp64 linear (alone, and for both random projections around the pinned
+attention oracle), and identity projections that reduce the block to that
+attention oracle.
 """
 import numpy as np
 import pytest
@@ -96,3 +97,23 @@ def test_projected_qkv_orders_q_k_v_then_heads():
             assert qkv[0, 1, c, h, 5] == 100 * c + 10 * h + 1
             assert qkv[0, 0, c, h, 5] == 0 and qkv[0, 2, c, h, 5] == 0
     assert np.count_nonzero(qkv) == 6
+
+
+@pytest.mark.parametrize("mode", ["frame", "global", "register"])
+def test_block_matches_torch_linear_around_the_attention_core(mode):
+    """Random (non-symmetric) projections: torch's fp64 linear for both maps around
+    the pinned attention oracle.  An untransposed output weight or the q/k/v
+    channel blocks taken in another order change the result."""
+    shape = W.Shape(S=2, T=11, H=2, n_special=3, grid_h=2, grid_w=4)
+    block = W.make_block_inputs(shape, 6)
+    q = oracle.register_tokens(shape) if mode == "register" else None
+    x = torch.from_numpy(oracle.bf16_to_f64(block["x"]))
+    qkv = torch.nn.functional.linear(x, torch.from_numpy(oracle.bf16_to_f64(block["w_qkv"])),
+                                     torch.from_numpy(block["b_qkv"].astype(np.float64)))
+    inputs = {"qkv_f64": qkv.numpy().reshape(shape.S, shape.T, 3, shape.H, 64),
+              **{k: block[k] for k in ("q_gamma", "q_beta", "k_gamma", "k_beta")}}
+    a = oracle.attn_mode(mode, shape, inputs, q)
+    want = torch.nn.functional.linear(torch.from_numpy(a.reshape(a.shape[0], -1)),
+                                      torch.from_numpy(oracle.bf16_to_f64(block["w_out"])),
+                                      torch.from_numpy(block["b_out"].astype(np.float64))).numpy()
+    np.testing.assert_allclose(oracle.attention_block(mode, shape, block, q), want, rtol=1e-11, atol=1e-11)
