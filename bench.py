@@ -458,7 +458,9 @@ def run_ours(args):
 def run_sharded(args):
     """--sharded: one scene (the 100-frame global workload) split across the ranks by frames; every step is
     query-sharded global attention (vit_attention_b200.sharded.global_attention_sharded: the rank's prologue,
-    one NCCL all-gather each of the normalised keys and of the values, the rank's core over all keys).
+    one NCCL all-gather each of the normalised keys and of the values, then the rank's core over all keys; with
+    --overlap the gather runs on a side stream beside the core over the rank's own keys, then the core over the
+    other ranks' keys merges with that).
     `value` = the scene's algorithmic flops per step / the max-over-ranks time ("scaling": "strong"); `e2e`
     adds, every step, the H2D of the rank's qkv frames from pinned host memory and the D2H of its output
     rows (serialised with the step on the rank's stream)."""
@@ -466,7 +468,7 @@ def run_sharded(args):
     import torch
     import torch.distributed as dist
     import vit_attention_b200 as V
-    from vit_attention_b200.sharded import global_attention_sharded
+    from vit_attention_b200.sharded import global_attention_sharded, overlapped
 
     rank, world, local = dist_env()
     if world > 1:
@@ -488,7 +490,7 @@ def run_sharded(args):
 
     def step():
         global_attention_sharded(shape, qkv, g["q_gamma"], g["q_beta"], g["k_gamma"], g["k_beta"], out, ws,
-                                 stream=stream)
+                                 stream=stream, overlap=args.overlap)
 
     for _ in range(args.warmup):
         step()
@@ -527,10 +529,18 @@ def run_sharded(args):
     torch.cuda.synchronize(device)
     barrier(device)
     e2e_ms = reduce_max(e0.elapsed_time(e1), device)
-    # the scene's per-rank core alone (the all-gather and the prologue excluded), for the roofline
+    # the scene's per-rank core alone (the all-gather and the prologue excluded), for the roofline; overlapped,
+    # the own keys' launch and the other ranks' launch with the merge
     k_send, v_send, k_all, v_all = V.vggt_attn_shard_buffers(shape, world, ws)
-    core_ms = reduce_max(cuda_time_ms(lambda: V.vggt_attn_global_shard_core(shape, world, out, ws, None, stream),
-                                      stream, max(3, args.steps)), device)
+    split = overlapped(world, args.overlap)
+    if split:
+        def core():
+            V.vggt_attn_global_shard_core_local(shape, world, ws, None, stream)
+            V.vggt_attn_global_shard_core_remote(shape, world, rank, out, ws, None, stream)
+    else:
+        def core():
+            V.vggt_attn_global_shard_core(shape, world, out, ws, None, stream)
+    core_ms = reduce_max(cuda_time_ms(core, stream, max(3, args.steps)), device)
     peaks, peak_src = load_peaks()
     peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
     core_tflops = flops / world / (core_ms / 1000.0) / 1e12
@@ -541,7 +551,8 @@ def run_sharded(args):
     if rank != 0:
         return 0
     cfg = headline_config(w, world)
-    cfg["parallelism"] = f"query-sharded x{world} over frames, NCCL all-gather of k and v (strong)"
+    cfg["parallelism"] = (f"query-sharded x{world} over frames, NCCL all-gather of k and v "
+                          f"{'beside the own keys attention' if split else 'then the core'} (strong)")
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic", "config": cfg,
@@ -550,10 +561,13 @@ def run_sharded(args):
                     "ms_per_step": e2e_ms / args.steps, "per_rank_bytes": True},
             "roofline": {"bound": "tensor", "achieved": core_tflops, "peak": peak, "unit": "TFLOP/s",
                          "frac": core_tflops / peak, "traffic": None,
-                         "kernel": "vggt::attn_core_kernel<CoreCfg<2, false, true>> (one rank's queries, all keys)",
+                         "kernel": ("vggt::attn_core_kernel<CoreCfg<2, false, true, false, 1>> + "
+                                    "attn_core_ranks_kernel<CoreCfg<2, false, true, true, 2>> (one rank's queries: "
+                                    "own keys, then the other ranks' keys with the merge)" if split else
+                                    "vggt::attn_core_kernel<CoreCfg<2, false, true>> (one rank's queries, all keys)"),
                          "kernel_ms": core_ms, "peak_source": f"{peak_src} bf16_tflops_sustained",
                          "allgather_bytes_per_rank": gather_bytes},
-            "gpu_launches": 2 * args.steps, "clocks": clk, "cpu_baseline": None}
+            "gpu_launches": (3 if split else 2) * args.steps, "clocks": clk, "cpu_baseline": None}
     print(json.dumps(line), flush=True)
     return 0
 
@@ -647,6 +661,19 @@ def sharded_timings(V, device, stream, qkv, prm, global_ms):
                                  "speedup_vs_1gpu_global": global_ms / (t_pro + t_core),
                                  "allgather_bytes_per_rank": gather_bytes,
                                  "allgather_ms_at_770GBs": gather_bytes / 770e9 * 1e3}
+        if world >= 2:
+            # overlapped form: the own keys' core (beside the all-gather), then the other ranks' keys with the merge
+            local_core = lambda: V.vggt_attn_global_shard_core_local(local, world, ws, None, stream)  # noqa: E731
+            remote_core = lambda: V.vggt_attn_global_shard_core_remote(local, world, 0, out_r, ws, None, stream)  # noqa: E731
+            local_core()
+            remote_core()
+            t_local = cuda_time_ms(local_core, stream, 3)
+            t_remote = cuda_time_ms(remote_core, stream, 3)
+            assert V.vggt_attn_read_status(ws, stream) == 0
+            gather_ms = gather_bytes / 770e9 * 1e3
+            res[f"world_{world}"].update({"rank_core_local_ms": t_local, "rank_core_remote_ms": t_remote,
+                                          "rank_core_split_ms": t_local + t_remote,
+                                          "allgather_exposed_ms_at_770GBs": max(0.0, gather_ms - t_local)})
         del ws, out_r
     return res
 
@@ -975,6 +1002,9 @@ def main():
     ap.add_argument("--sharded", action="store_true",
                     help="one 100-frame scene split across the ranks by frames: query-sharded global attention with "
                          "an NCCL all-gather of the keys and values (strong scaling; the ranks must divide 100)")
+    ap.add_argument("--overlap", action="store_true",
+                    help="with --sharded: the all-gather on a side stream beside the core over the rank's own keys, "
+                         "then the other ranks' keys with a merge (2 to 9 ranks)")
     ap.add_argument("--one", choices=("frame", "global", "register"), default=None,
                     help="run only this mode on --workload's shape (--frames, --calls, --block, --sga, --desc) and "
                          "exit: a small case for ncu")

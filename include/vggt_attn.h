@@ -414,7 +414,8 @@ int vggt_attn_host_pipeline(int mode, const vggt_attn_shape* shape, int n_items,
  * every query row sees the same keys in the same 64-key steps).  world = 1
  * is plain global attention with the copies in between.  The workspace
  * (vggt_attn_shard_workspace_size bytes) holds the status word, the q plane,
- * both send buffers and both gathered buffers; the first kernel of call 1
+ * both send buffers, both gathered buffers and the partial softmax state of
+ * the overlapped form (below); the first kernel of call 1
  * clears the status word.  Calls are asynchronous on cuda_stream, validate
  * every argument before enqueueing anything and allocate nothing;
  * vggt_attn_shard_buffers does no device work. */
@@ -443,6 +444,36 @@ int vggt_attn_global_shard_prologue(const vggt_attn_shape* shape, int world, con
                                     void* workspace, size_t workspace_bytes, void* cuda_stream);
 int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int world, void* out,
                                 void* workspace, size_t workspace_bytes, void* cuda_stream);
+/* Overlapped form of step 3, so that the all-gather runs beside attention:
+ *
+ *   3a. vggt_attn_global_shard_core_local (right after the prologue, on the
+ *       compute stream, while the all-gather of step 2 runs on another
+ *       stream): the rank's queries over its OWN keys and values, read from
+ *       k_send / v_send.  Writes no output: it leaves each query row's
+ *       softmax state over those keys in the workspace (fp32: the 64
+ *       unnormalised sums of 2^(s - m) v, their weight sum and the reference
+ *       max m; the workspace of vggt_attn_shard_workspace_size holds it).
+ *       Reads nothing the all-gather writes and writes nothing it reads.
+ *   3b. vggt_attn_global_shard_core_remote (after the all-gather has
+ *       completed): the queries over the other world - 1 ranks' blocks of
+ *       k_all / v_all (rank `rank`'s own block is skipped), merging the state
+ *       3a left (both scaled to the larger reference max and added) before
+ *       the division by the row sum; writes out as step 3 does.
+ *
+ * The softmax over the union of the two key sets is the attention over all
+ * keys (VGGT-Omega Aggregator explainer, section 3: global attention over
+ * every frame's tokens); the result equals step 3's to rounding (different
+ * 64-key step boundaries and the fp32 merge), not bit for bit.  3b needs
+ * 2 <= world <= 9 (one tensor map per remote rank) and 0 <= rank < world,
+ * else VGGT_ATTN_ERR_UNSUPPORTED_SHAPE / VGGT_ATTN_ERR_INVALID_ARG; with one
+ * rank call step 3.  3b must follow 3a of the same workspace on the GPU
+ * (same stream, or an event between them).  Cost: the two launches take
+ * 4-7 % longer than step 3's one launch (100-frame scene, 2-5 ranks, B200),
+ * so the overlap pays only where the all-gather takes longer than that. */
+int vggt_attn_global_shard_core_local(const vggt_attn_shape* shape, int world, void* workspace,
+                                      size_t workspace_bytes, void* cuda_stream);
+int vggt_attn_global_shard_core_remote(const vggt_attn_shape* shape, int world, int rank, void* out,
+                                       void* workspace, size_t workspace_bytes, void* cuda_stream);
 
 /* ------------------------------------------------------------------------
  * Camera-head trunk (VGGT-Omega Aggregator explainer, section 4: the camera

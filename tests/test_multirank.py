@@ -1,6 +1,8 @@
 """Host-side logic of the multi-GPU bench path, run as 2 gloo ranks on CPU:
 each rank gets its own independent workload copy (weak scaling, no data
-exchange) and the timed region is the max over ranks."""
+exchange) and the timed region is the max over ranks; the exchange step of
+query-sharded global attention (the all-gather in rank order) and the order of
+the overlapped form's host steps (streams and library calls recorded by fakes)."""
 import os
 import socket
 
@@ -157,3 +159,86 @@ def test_sharded_scene_gathers_the_whole_scene_on_every_rank():
     for r in range(world):
         assert res[r][1] and res[r][2]
         assert res[r][3] == 1.0
+
+
+# ---------------------------------------------------------------- overlapped form: the order of the host's steps
+class _Stream:
+    def __init__(self, name, log):
+        self.name, self.log, self.device = name, log, "cuda:0"
+
+    def wait_stream(self, other):
+        self.log.append(("wait", self.name, other.name))
+
+
+class _Buf:
+    def __init__(self, name, log):
+        self.name, self.log = name, log
+
+    def copy_(self, src):
+        self.log.append(("copy", self.name, src.name))
+
+
+def _fake_sharded(monkeypatch, world, rank):
+    """sharded.global_attention_sharded with the library calls, the streams and the process group replaced
+    by recorders: returns (the call, the log).  Each log entry names the stream it was enqueued on."""
+    V = pytest.importorskip("vit_attention_b200", reason="libvggt_attn.so is not built")
+    import contextlib
+    import torch
+    import torch.distributed as dist
+    from vit_attention_b200 import sharded
+    log = []
+    main, comm = _Stream("main", log), _Stream("comm", log)
+    current = [main]
+
+    @contextlib.contextmanager
+    def on(stream):
+        prev = current[0]
+        current[0] = stream
+        try:
+            yield
+        finally:
+            current[0] = prev
+
+    bufs = [_Buf(n, log) for n in ("k_send", "v_send", "k_all", "v_all")]
+    monkeypatch.setattr(torch.cuda, "stream", on)
+    monkeypatch.setattr(torch.cuda, "current_stream", lambda *a: current[0])
+    monkeypatch.setattr(sharded, "_side_stream", lambda device: comm)
+    monkeypatch.setattr(dist, "is_initialized", lambda: True)
+    monkeypatch.setattr(dist, "get_world_size", lambda group=None: world)
+    monkeypatch.setattr(dist, "get_rank", lambda group=None: rank)
+    monkeypatch.setattr(sharded, "gather_kv", lambda *a, **k: log.append(("gather", current[0].name)))
+    monkeypatch.setattr(V, "vggt_attn_shard_buffers", lambda *a, **k: bufs)
+    monkeypatch.setattr(V, "vggt_attn_global_shard_prologue", lambda *a, stream=None, **k: log.append(("prologue", stream.name)))
+    monkeypatch.setattr(V, "vggt_attn_global_shard_core", lambda *a, stream=None, **k: log.append(("core", stream.name)))
+    monkeypatch.setattr(V, "vggt_attn_global_shard_core_local",
+                        lambda *a, stream=None, **k: log.append(("core_local", stream.name)))
+    monkeypatch.setattr(V, "vggt_attn_global_shard_core_remote",
+                        lambda shape, w, r, *a, stream=None, **k: log.append(("core_remote", stream.name, r)))
+
+    def call(**kw):
+        sharded.global_attention_sharded("shape", None, None, None, None, None, "out", "ws", stream=main, **kw)
+        return log
+    return call
+
+
+@pytest.mark.parametrize("world,rank", [(2, 1), (8, 3), (9, 8)])
+def test_overlapped_steps_gather_beside_the_own_keys_core(monkeypatch, world, rank):
+    log = _fake_sharded(monkeypatch, world, rank)(overlap=True)
+    assert log == [("prologue", "main"),
+                   ("wait", "comm", "main"),          # the side stream waits for the send buffers
+                   ("gather", "comm"),                # the all-gather on the side stream ...
+                   ("core_local", "main"),            # ... beside the own keys' core, which does not wait for it
+                   ("wait", "main", "comm"),          # the remote keys' core waits for the gather
+                   ("core_remote", "main", rank)]
+
+
+@pytest.mark.parametrize("world,overlap", [(2, None), (2, False), (10, True)])
+def test_gather_then_one_core_without_overlap(monkeypatch, world, overlap):
+    kw = {} if overlap is None else {"overlap": overlap}      # the default is the one-pass core
+    log = _fake_sharded(monkeypatch, world, 0)(**kw)
+    assert log == [("prologue", "main"), ("gather", "main"), ("core", "main")]
+
+
+def test_one_rank_copies_instead_of_gathering(monkeypatch):
+    log = _fake_sharded(monkeypatch, 1, 0)()
+    assert log == [("prologue", "main"), ("copy", "k_all", "k_send"), ("copy", "v_all", "v_send"), ("core", "main")]

@@ -97,6 +97,97 @@ def test_single_rank_helper_without_process_group():
     assert torch.equal(out.view(torch.int16), _run_global(shape, dev).view(torch.int16))
 
 
+# ------------------------------------------------------------------ overlapped form (own keys, then the others')
+def _run_overlapped(shape, dev, world):
+    """Every rank's prologue and own-keys core (the launch that runs beside the all-gather), the gather
+    emulated with device copies, then each rank's core over the other ranks' keys with the merge."""
+    import dataclasses
+    import torch
+    import vit_attention_b200 as V
+    local = dataclasses.replace(shape, S=shape.S // world)
+    wss, sends = [], []
+    for r in range(world):
+        ws = torch.empty(V.vggt_attn_shard_workspace_size(local, world), dtype=torch.uint8, device="cuda")
+        V.vggt_attn_global_shard_prologue(local, world, dev["qkv"][r * local.S:(r + 1) * local.S], dev["q_gamma"],
+                                          dev["q_beta"], dev["k_gamma"], dev["k_beta"], ws)
+        V.vggt_attn_global_shard_core_local(local, world, ws)
+        wss.append(ws)
+        sends.append(V.vggt_attn_shard_buffers(local, world, ws)[:2])
+    k_cat = torch.cat([k for k, _ in sends])
+    v_cat = torch.cat([v for _, v in sends])
+    outs = []
+    for r in range(world):
+        _, _, k_all, v_all = V.vggt_attn_shard_buffers(local, world, wss[r])
+        k_all.copy_(k_cat)
+        v_all.copy_(v_cat)
+        out = torch.zeros((local.S, local.T, local.H, 64), dtype=torch.bfloat16, device="cuda")
+        V.vggt_attn_global_shard_core_remote(local, world, r, out, wss[r])
+        assert V.vggt_attn_read_status(wss[r]) == 0
+        outs.append(out)
+    return torch.cat(outs)
+
+
+# ragged local token counts (136, 634, 14) and the largest world (8 remote rank maps)
+OVERLAP = [(shp(6, 4, 5, 7, 9), 3), (shp(4, 2, 17, 10, 30), 2), (shp(8, 2, 5, 3, 4), 8), (shp(9, 2, 5, 3, 4), 9)]
+
+
+@pytest.mark.parametrize("shape,world", OVERLAP, ids=[f"S{s.S}T{s.T}H{s.H}-w{w}" for s, w in OVERLAP])
+def test_overlapped_ranks_match_oracle(shape, world):
+    """Every query row against the fp64 oracle; and against the one-pass gathered core to bf16 rounding
+    (the key order and the 64-key step boundaries differ, so not bit for bit)."""
+    import torch
+    x = W.make_random_inputs(shape, 240 + shape.T + world)
+    dev = _dev(x)
+    got = _run_overlapped(shape, dev, world)
+    q = query_sample("global", shape, 1 << 62, 0)
+    assert_close(rows(got, shape, q), O.attn_global(shape, x, q), f"overlapped sharded global, {world} ranks")
+    one_pass = _run_sharded(shape, dev, world).float()
+    diff = (got.float() - one_pass).abs().max().item()
+    assert diff <= 2.0 ** -5, f"overlapped vs one-pass core: max |diff| = {diff}"
+
+
+def test_overlapped_workload2_four_ranks_against_oracle():
+    w = W.workload(2)                                  # 24 frames x 1031 tokens, 16 heads
+    x = W.make_inputs(w)
+    got = _run_overlapped(w.shape, _dev(x), 4)
+    q = query_sample("global", w.shape, 512, w.seed + 1)
+    assert_close(rows(got, w.shape, q), O.attn_global(w.shape, x, q), "overlapped sharded global, 4 ranks")
+
+
+def test_overlapped_merge_with_distant_maxima():
+    """Rank 0's keys point along -u, rank 1's along +u, and the queries alternate between +u and -u, so for
+    every rank some rows find their maxima among their own keys and others among the other rank's, 15-20
+    units (base 2) above the rest: the merge scales one side by about 2^-18.  The bf16 storage points alone
+    err by 1.8e-3 (max-abs) / 3.5e-3 (rel.) on these inputs (CPU emulation, as in test_parity_gpu); a merge
+    that scaled the wrong side would be off by O(1)."""
+    shape = W.Shape(S=4, T=40, H=2, n_special=40, grid_h=0, grid_w=1)
+    x = W.make_random_inputs(shape, 250)
+    qkv = O.bf16_to_f64(x["qkv"])
+    u = np.random.default_rng(251).standard_normal(64)
+    u -= u.mean()
+    u /= np.linalg.norm(u)
+    for s in range(shape.S):
+        qkv[s, :, 1] += (16.0 if s >= shape.S // 2 else -16.0) * u
+        qkv[s, :, 0] += np.where(np.arange(shape.T) % 2 == 0, 16.0, -16.0)[:, None, None] * u
+    x["qkv"] = W.f32_to_bf16_bits(qkv.astype(np.float32))
+    got = _run_overlapped(shape, _dev(x), 2)
+    q = np.arange(shape.S * shape.T)
+    assert_close(rows(got, shape, q), O.attn_global(shape, x, q), "overlapped sharded global, distant maxima")
+
+
+def test_overlapped_remote_rejects_bad_world_and_rank():
+    import dataclasses
+    import torch
+    import vit_attention_b200 as V
+    shape = shp(10, 2, 5, 3, 4)
+    for world, rank in ((1, 0), (10, 0), (2, 2), (2, -1)):
+        local = dataclasses.replace(shape, S=shape.S // world)
+        ws = torch.empty(V.vggt_attn_shard_workspace_size(local, world), dtype=torch.uint8, device="cuda")
+        out = torch.zeros((local.S, local.T, local.H, 64), dtype=torch.bfloat16, device="cuda")
+        with pytest.raises(RuntimeError):
+            V.vggt_attn_global_shard_core_remote(local, world, rank, out, ws)
+
+
 # ------------------------------------------------------------------ fused form (keys read in place)
 def _fused_emulated(shape, dev, world):
     """All ranks in this process: W prologues into W workspaces, then each rank's core reads the W send

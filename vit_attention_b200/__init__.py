@@ -98,6 +98,8 @@ _SIGNATURES = {
                                        ctypes.POINTER(_vp), ctypes.POINTER(_vp)]),
     "vggt_attn_global_shard_prologue": (_int, [_shape_p, _int, _vp, _fp, _fp, _fp, _fp, _vp, _sz, _vp]),
     "vggt_attn_global_shard_core": (_int, [_shape_p, _int, _vp, _vp, _sz, _vp]),
+    "vggt_attn_global_shard_core_local": (_int, [_shape_p, _int, _vp, _sz, _vp]),
+    "vggt_attn_global_shard_core_remote": (_int, [_shape_p, _int, _int, _vp, _vp, _sz, _vp]),
     "vggt_attn_shard_fused_workspace_size": (_sz, [_shape_p]),
     "vggt_attn_global_shard_core_peers": (_int, [_shape_p, _int, ctypes.POINTER(_vp), ctypes.POINTER(_vp), _vp,
                                                  _vp, _sz, _vp]),
@@ -406,6 +408,23 @@ def vggt_attn_global_shard_core(shape, world, out, workspace, workspace_bytes=No
     rc = _lib.vggt_attn_global_shard_core(ctypes.byref(make_shape(shape)), world, _ptr(out), _ptr(workspace),
                                           _nbytes(workspace, workspace_bytes), _stream(stream))
     _check(rc, "vggt_attn_global_shard_core")
+
+
+def vggt_attn_global_shard_core_local(shape, world, workspace, workspace_bytes=None, stream=None):
+    """Overlapped form, first half: the rank's queries over its own keys (send buffers) into the workspace's
+    partial softmax state; runs while the all-gather fills the gathered buffers."""
+    rc = _lib.vggt_attn_global_shard_core_local(ctypes.byref(make_shape(shape)), world, _ptr(workspace),
+                                                _nbytes(workspace, workspace_bytes), _stream(stream))
+    _check(rc, "vggt_attn_global_shard_core_local")
+
+
+def vggt_attn_global_shard_core_remote(shape, world, rank, out, workspace, workspace_bytes=None, stream=None):
+    """Overlapped form, second half (after the all-gather): the other ranks' keys, merged with the partial
+    state of vggt_attn_global_shard_core_local, into out."""
+    rc = _lib.vggt_attn_global_shard_core_remote(ctypes.byref(make_shape(shape)), world, rank, _ptr(out),
+                                                 _ptr(workspace), _nbytes(workspace, workspace_bytes),
+                                                 _stream(stream))
+    _check(rc, "vggt_attn_global_shard_core_remote")
 
 
 def vggt_attn_host_pipeline_workspace_size(shape, mode) -> int:

@@ -6,7 +6,10 @@
 // describes NQ = 2).  Configurations (CoreCfg): SGA adds the subsampled global
 // attention terms in the epilogue, KTM reads keys token-major like values,
 // RANKS reads the keys and values of several ranks' buffers in turn
-// (attn_core_ranks_kernel, query-sharded global attention):
+// (attn_core_ranks_kernel, query-sharded global attention), PART splits one
+// row's keys over two launches (the first leaves its softmax state, the
+// second merges it; query-sharded global attention with the all-gather
+// overlapped):
 //   O = softmax(Q K^T) V   over the problem's L keys.  Q arrives scaled by
 //   softmax_scale*log2(e) from the prologue, so scores are in base 2.
 // (VGGT-Omega Aggregator explainer, section 3: the frame / global / register
@@ -97,6 +100,13 @@ struct CoreParams {
   SgaParams sga;      // SGA configuration only
   int rank_tokens;    // per-rank key blocks (RANKS configuration): keys per rank,
   int rank_steps;     // and 64-key steps per rank (the last one ragged)
+  // Softmax state of row i of head h over part of the keys (PART
+  // configurations): part_o[(h L + i) 64 + d] = sum over those keys of
+  // 2^(s - m) v_d and part_ml[2 (h L + i)] = {sum of 2^(s - m), m}, m the
+  // row's reference max (base-2 scores); part_rows = H L.
+  float* part_o;
+  float* part_ml;
+  long long part_rows;
 };
 
 // Keys and values of a query-sharded global attention, one tensor map per
@@ -129,7 +139,7 @@ constexpr uint32_t POLY_PAIR_MASK = 0x80u;
 // shape instead (attention_frame_persistent.cuh): its CTAs take tile after
 // tile and start the next tile's products during the last one's epilogue,
 // 2 % faster on the 500-frame workload.
-template <int NQ_, bool SGA_ = false, bool KTM_ = false, bool RANKS_ = false>
+template <int NQ_, bool SGA_ = false, bool KTM_ = false, bool RANKS_ = false, int PART_ = 0>
 struct CoreCfg {
   static constexpr int NQ = NQ_;
   static constexpr bool SGA = SGA_;   // subsampled global attention epilogue
@@ -140,6 +150,12 @@ struct CoreCfg {
   // block starts a new 64-key step and its last step is masked to its length.
   static constexpr bool RANKS = RANKS_;
   static_assert(!RANKS_ || KTM_, "rank blocks are token-major");
+  // Epilogue: 0 writes softmax(Q K^T) V as bf16; 1 writes the rows' softmax
+  // state over this launch's keys (CoreParams::part_*) instead; 2 merges that
+  // state with its own before writing bf16, so that two launches over
+  // disjoint key sets give the attention over their union.
+  static constexpr int PART = PART_;
+  static_assert(PART_ >= 0 && PART_ <= 2 && !(SGA_ && PART_), "epilogue configuration");
   static constexpr int CTAS_PER_SM = NQ_ == 2 ? 1 : 2;
   static constexpr int STAGES = NQ_ == 2 ? 8 : 5;
   static constexpr int OFF_Q = 0;                                  // NQ tiles
@@ -498,8 +514,43 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     tmem_ld1(o_addr + D, osum);
     tmem_wait_ld();
     const int i = q0 + tile * BM + row;
-    if (i < p.L) {
+    if (C::PART == 1 && i < p.L) {
+      const long long pr = static_cast<long long>(h) * p.L + i;
+      if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x910u)) {
+        float4* dst = reinterpret_cast<float4*>(p.part_o + pr * D);
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            dst[c * 8 + v] = make_float4(__uint_as_float(orr[c][4 * v]), __uint_as_float(orr[c][4 * v + 1]),
+                                         __uint_as_float(orr[c][4 * v + 2]), __uint_as_float(orr[c][4 * v + 3]));
+        reinterpret_cast<float2*>(p.part_ml)[pr] = make_float2(__uint_as_float(osum), m_run);
+      }
+    } else if (i < p.L) {
       if constexpr (C::SGA) sga_extra_terms(p, h, i, m_run, orr, osum);
+      if constexpr (C::PART == 2) {
+        // The other launch's state over its keys, both relative to their own
+        // reference max: scale each to the larger one and add.
+        const long long pr = static_cast<long long>(h) * p.L + i;
+        if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x918u)) {
+          const float2 ml = reinterpret_cast<const float2*>(p.part_ml)[pr];
+          const float m = fmaxf(m_run, ml.y);
+          const float a_own = ex2_approx(m_run - m), a_part = ex2_approx(ml.y - m);
+          const float4* src = reinterpret_cast<const float4*>(p.part_o + pr * D);
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              const float4 o1 = src[c * 8 + v];
+              uint32_t* o = &orr[c][4 * v];
+              o[0] = __float_as_uint(__uint_as_float(o[0]) * a_own + o1.x * a_part);
+              o[1] = __float_as_uint(__uint_as_float(o[1]) * a_own + o1.y * a_part);
+              o[2] = __float_as_uint(__uint_as_float(o[2]) * a_own + o1.z * a_part);
+              o[3] = __float_as_uint(__uint_as_float(o[3]) * a_own + o1.w * a_part);
+            }
+          osum = __float_as_uint(__uint_as_float(osum) * a_own + ml.x * a_part);
+        }
+      }
       const float inv = 1.f / __uint_as_float(osum);
       const long long out_row = static_cast<long long>(b) * p.out_T +
                                 static_cast<long long>(i / p.out_group) * p.out_T + (i % p.out_group);

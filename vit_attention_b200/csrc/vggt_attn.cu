@@ -1339,6 +1339,8 @@ struct ShardLayout {
   uint16_t* v_send;
   uint16_t* k_all;          // [world L][H][64]
   uint16_t* v_all;
+  float* part_o;            // [H][L][64]: softmax state over the rank's own keys (overlapped form)
+  float* part_ml;           // [H][L][2]
   long long L, Lk;
   size_t bytes;
 };
@@ -1363,6 +1365,10 @@ ShardLayout shard_layout(const vggt_attn_shape* s, int world, void* ws) {
   off += align256(S.Lk * row);
   S.v_all = reinterpret_cast<uint16_t*>(base + off);
   off += align256(S.Lk * row);
+  S.part_o = reinterpret_cast<float*>(base + off);
+  off += align256(static_cast<size_t>(s->H) * S.L * 64 * sizeof(float));
+  S.part_ml = reinterpret_cast<float*>(base + off);
+  off += align256(static_cast<size_t>(s->H) * S.L * 2 * sizeof(float));
   S.w.bytes = off;
   S.bytes = off;
   return S;
@@ -1470,6 +1476,108 @@ extern "C" int vggt_attn_global_shard_core(const vggt_attn_shape* shape, int wor
   p.timeout_ns = kDefaultTimeoutNs;
   ModeGeometry g{1, L.L, L.L, 2};
   return launch_core_cfg<vggt::CoreCfg<2, false, true>>(g, shape->H, mq, mk, mv, p, static_cast<cudaStream_t>(cuda_stream));
+}
+
+// Overlapped form: the rank's own keys first (from its send buffers, while the
+// all-gather runs), then the other ranks' blocks of the gathered buffers with
+// the first launch's softmax state merged in the epilogue.
+namespace {
+
+bool shard_q_map(CUtensorMap* mq, const ShardLayout& L, long long H) {
+  const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(L.L), static_cast<cuuint64_t>(H)};
+  const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(L.L) * 128};
+  const cuuint32_t box_q[3] = {64, vggt::core::BM, 1};
+  return make_map(mq, L.w.q, 3, dims, strides, box_q);
+}
+
+// keys or values of one rank, [L][H][64] as (dim, head, token, 1); rows past L read as zeros
+bool shard_block_map(CUtensorMap* m, const void* base, const ShardLayout& L, long long H) {
+  const cuuint64_t dims[4] = {64, static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(L.L), 1};
+  const cuuint64_t strides[3] = {128, static_cast<cuuint64_t>(H) * 128, static_cast<cuuint64_t>(L.L) * H * 128};
+  const cuuint32_t box[4] = {64, 1, vggt::core::BN, 1};
+  return make_map(m, base, 4, dims, strides, box);
+}
+
+vggt::CoreParams shard_core_params(const vggt_attn_shape* shape, const ShardLayout& L, void* out) {
+  vggt::CoreParams p{};
+  p.L = static_cast<int>(L.L);
+  p.H = shape->H;
+  p.B = 1;
+  p.out_T = shape->T;
+  p.out_group = static_cast<int>(L.L);
+  p.out = static_cast<uint16_t*>(out);
+  p.out_elems = out ? static_cast<long long>(shape->S) * shape->T * shape->H * 64 : 0;
+  p.status = L.w.status;
+  p.timeout_ns = kDefaultTimeoutNs;
+  p.part_o = L.part_o;
+  p.part_ml = L.part_ml;
+  p.part_rows = static_cast<long long>(shape->H) * L.L;
+  return p;
+}
+
+}  // namespace
+
+extern "C" int vggt_attn_global_shard_core_local(const vggt_attn_shape* shape, int world, void* workspace,
+                                                 size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes))) return rc;
+  if ((rc = check_device())) return rc;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  CUtensorMap mq, mk, mv;
+  if (!shard_q_map(&mq, L, shape->H) || !shard_block_map(&mk, L.k_send, L, shape->H) ||
+      !shard_block_map(&mv, L.v_send, L, shape->H))
+    return VGGT_ATTN_ERR_CUDA;
+  vggt::CoreParams p = shard_core_params(shape, L, nullptr);
+  p.Lk = static_cast<int>(L.L);
+  ModeGeometry g{1, L.L, L.L, 2};
+  return launch_core_cfg<vggt::CoreCfg<2, false, true, false, 1>>(g, shape->H, mq, mk, mv, p,
+                                                                  static_cast<cudaStream_t>(cuda_stream));
+}
+
+extern "C" int vggt_attn_global_shard_core_remote(const vggt_attn_shape* shape, int world, int rank, void* out,
+                                                  void* workspace, size_t workspace_bytes, void* cuda_stream) {
+  int rc = check_shard_shape(shape, world);
+  if (rc) return rc;
+  if (world < 2 || world - 1 > vggt::kMaxRankMaps) return VGGT_ATTN_ERR_UNSUPPORTED_SHAPE;
+  if (rank < 0 || rank >= world) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_shard_ws(shape, world, workspace, workspace_bytes))) return rc;
+  if (!out) return VGGT_ATTN_ERR_INVALID_ARG;
+  if (!aligned(out, 16)) return VGGT_ATTN_ERR_MISALIGNED;
+  const size_t out_bytes = static_cast<size_t>(shape->S) * shape->T * shape->H * 128;
+  if (overlaps(out, out_bytes, workspace, workspace_bytes)) return VGGT_ATTN_ERR_INVALID_ARG;
+  if ((rc = check_device())) return rc;
+  using C = vggt::CoreCfg<2, false, true, true, 2>;
+  const ShardLayout L = shard_layout(shape, world, workspace);
+  const long long H = shape->H;
+  CUtensorMap mq;
+  if (!shard_q_map(&mq, L, H)) return VGGT_ATTN_ERR_CUDA;
+  vggt::RankMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  const size_t block = static_cast<size_t>(L.L) * H * 64;   // elements of one rank's block
+  for (int q = 0, n = 0; q < world; ++q) {
+    if (q == rank) continue;
+    if (!shard_block_map(&maps.k[n], L.k_all + q * block, L, H) ||
+        !shard_block_map(&maps.v[n], L.v_all + q * block, L, H))
+      return VGGT_ATTN_ERR_CUDA;
+    ++n;
+  }
+  const int spr = static_cast<int>((L.L + vggt::core::BN - 1) / vggt::core::BN);
+  vggt::CoreParams p = shard_core_params(shape, L, out);
+  p.Lk = (world - 1) * spr * vggt::core::BN;   // n_kv = (world - 1) * spr steps
+  p.rank_tokens = static_cast<int>(L.L);
+  p.rank_steps = spr;
+  if (cudaFuncSetAttribute(vggt::attn_core_ranks_kernel<C>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           C::SMEM_ALLOC) != cudaSuccess)
+    return VGGT_ATTN_ERR_CUDA;
+  cudaFuncAttributes fa;   // the register split assumes the compiled count (see launch_core_cfg)
+  if (cudaFuncGetAttributes(&fa, vggt::attn_core_ranks_kernel<C>) != cudaSuccess || fa.numRegs < C::REGS_AT_LAUNCH)
+    return VGGT_ATTN_ERR_CUDA;
+  const long long n_q = (L.L + 2 * vggt::core::BM - 1) / (2 * vggt::core::BM);
+  const dim3 grid(static_cast<unsigned>(n_q), static_cast<unsigned>(H), 1);
+  vggt::attn_core_ranks_kernel<C><<<grid, C::THREADS, C::SMEM_ALLOC, static_cast<cudaStream_t>(cuda_stream)>>>(
+      mq, maps, p);
+  return cudaGetLastError() == cudaSuccess ? VGGT_ATTN_OK : VGGT_ATTN_ERR_CUDA;
 }
 
 // ---------------------------------------------------------------------------

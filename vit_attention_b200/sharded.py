@@ -5,6 +5,17 @@ frame.  The exchange step is one all-gather of the normalised, rotated keys and
 one of the values (token-major, rank-major); the prologue before it and the
 attention core after it are the library's kernels (vggt_attn_global_shard_*).
 
+Overlapped (optional, 2 to 9 ranks): the all-gather runs on a side stream
+while the compute stream runs the core over the rank's own keys
+(vggt_attn_global_shard_core_local, which leaves each row's softmax state);
+after the gather the core runs over the other ranks' keys and merges that
+state (vggt_attn_global_shard_core_remote).  Only the gather time beyond the
+local keys' attention stays exposed, but the two launches cost 4-7 % more
+than the one-pass core (100-frame scene, 2-5 ranks, measured on a B200 with
+the ranks run one after another), more than an all-gather at NVLink 5
+speeds takes (1-4 % of the core), so it is off by default; it pays where the
+link is much slower than the core.
+
 The collective is the only data-path communication: head-sharded global
 attention (each rank a subset of heads over all tokens) needs none and is plain
 vggt_attn_global on a head slice of qkv.
@@ -28,26 +39,60 @@ def gather_kv(k_send, v_send, k_all, v_all, group=None) -> None:
     dist.all_gather_into_tensor(v_all, v_send, group=group)
 
 
+# The overlapped core's second launch reads one tensor map per remote rank.
+MAX_OVERLAP_WORLD = 9
+
+_side_streams = {}
+
+
+def _side_stream(device):
+    import torch
+    key = torch.device(device).index
+    if key not in _side_streams:
+        _side_streams[key] = torch.cuda.Stream(device=device)
+    return _side_streams[key]
+
+
+def overlapped(world: int, overlap: bool) -> bool:
+    """Whether global_attention_sharded runs the all-gather beside the local keys' attention."""
+    return overlap and 2 <= world <= MAX_OVERLAP_WORLD
+
+
 def global_attention_sharded(shape, qkv, q_gamma, q_beta, k_gamma, k_beta, out, workspace, group=None,
-                             stream=None) -> None:
+                             stream=None, overlap=False) -> None:
     """This rank's rows of global attention over the whole scene.
 
     shape: the LOCAL shape (S = frames on this rank, equal on every rank);
     qkv: this rank's frames, bf16 [S][T][3][H][64]; out: bf16 [S][T][H][64];
     workspace: uint8 tensor of vggt_attn_shard_workspace_size(shape, world) bytes.
+    overlap: run the all-gather on a side stream beside the attention over the
+    rank's own keys (2 to 9 ranks; equal to the one-pass result to rounding);
+    otherwise gather first, then one core over all keys (bit for bit
+    vggt_attn_global's rows).
     """
     import torch
     import torch.distributed as dist
     import vit_attention_b200 as V
     world = dist.get_world_size(group) if dist.is_initialized() else 1
+    rank = dist.get_rank(group) if dist.is_initialized() else 0
     V.vggt_attn_global_shard_prologue(shape, world, qkv, q_gamma, q_beta, k_gamma, k_beta, workspace,
                                       stream=stream)
     k_send, v_send, k_all, v_all = V.vggt_attn_shard_buffers(shape, world, workspace)
+    s = stream if stream is not None else torch.cuda.current_stream()
     if world == 1:
-        k_all.copy_(k_send)
-        v_all.copy_(v_send)
+        with torch.cuda.stream(s):
+            k_all.copy_(k_send)
+            v_all.copy_(v_send)
+    elif overlapped(world, overlap):
+        comm = _side_stream(s.device)
+        comm.wait_stream(s)                       # the prologue has written the send buffers
+        with torch.cuda.stream(comm):
+            gather_kv(k_send, v_send, k_all, v_all, group)
+        V.vggt_attn_global_shard_core_local(shape, world, workspace, stream=s)
+        s.wait_stream(comm)                       # every rank's keys and values are gathered
+        V.vggt_attn_global_shard_core_remote(shape, world, rank, out, workspace, stream=s)
+        return
     else:
-        s = stream if stream is not None else torch.cuda.current_stream()
         with torch.cuda.stream(s):
             gather_kv(k_send, v_send, k_all, v_all, group)
     V.vggt_attn_global_shard_core(shape, world, out, workspace, stream=stream)
