@@ -516,7 +516,7 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
     const int i = q0 + tile * BM + row;
     if (C::PART == 1 && i < p.L) {
       const long long pr = static_cast<long long>(h) * p.L + i;
-      if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x910u)) {
+      if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x930u)) {
         float4* dst = reinterpret_cast<float4*>(p.part_o + pr * D);
 #pragma unroll
         for (int c = 0; c < 2; ++c)
@@ -532,7 +532,7 @@ __device__ __forceinline__ void softmax_role(const CoreParams& p, const uint8_t*
         // The other launch's state over its keys, both relative to their own
         // reference max: scale each to the larger one and add.
         const long long pr = static_cast<long long>(h) * p.L + i;
-        if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x918u)) {
+        if (VGGT_DBG_BOUNDS(pr < p.part_rows, p.status, 0x938u)) {
           const float2 ml = reinterpret_cast<const float2*>(p.part_ml)[pr];
           const float m = fmaxf(m_run, ml.y);
           const float a_own = ex2_approx(m_run - m), a_part = ex2_approx(ml.y - m);
