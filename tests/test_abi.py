@@ -166,3 +166,34 @@ def test_empty_and_oversized_shapes_are_rejected_on_the_host(V):
     assert _call(V, f, huge, wsb=1 << 40) == V.ERR_UNSUPPORTED_SHAPE
     # zero heads
     assert _call(V, f, W.Shape(S=2, T=69, H=0, n_special=5, grid_h=8, grid_w=8), wsb=1 << 30) == V.ERR_UNSUPPORTED_SHAPE
+
+
+def test_overlapped_shard_core_validation_without_device(V):
+    """The overlapped sharded core's argument errors come back from the host before any device work, and
+    its workspace holds the partial softmax state (fp32 sums, row sum and max per row and head) on top of
+    the gathered buffers."""
+    import dataclasses
+    s = W.Shape(S=2, T=68, H=4, n_special=5, grid_h=7, grid_w=9)
+    lib = V.library()
+    shape = V.make_shape(s)
+    world = 2
+    L = s.S * s.T
+    wsb = V.vggt_attn_shard_workspace_size(s, world)
+    fused = V.vggt_attn_shard_fused_workspace_size(s)
+    assert wsb >= fused + 2 * world * L * s.H * 128 + s.H * L * (64 + 2) * 4
+    ws, out = 1 << 36, 1 << 34
+    local = lib.vggt_attn_global_shard_core_local
+    remote = lib.vggt_attn_global_shard_core_remote
+    assert local(ctypes.byref(shape), world, None, wsb, None) == V.ERR_INVALID_ARG
+    assert local(ctypes.byref(shape), world, ws + 16, wsb, None) == V.ERR_MISALIGNED
+    assert local(ctypes.byref(shape), world, ws, wsb - 1, None) == V.ERR_WORKSPACE_TOO_SMALL
+    assert local(ctypes.byref(shape), world, ws, fused, None) == V.ERR_WORKSPACE_TOO_SMALL   # the fused form's prefix only
+    one = V.make_shape(dataclasses.replace(s, S=4))
+    assert remote(ctypes.byref(one), 1, 0, out, ws, 1 << 32, None) == V.ERR_UNSUPPORTED_SHAPE   # nothing remote
+    assert remote(ctypes.byref(shape), 10, 0, out, ws, 1 << 32, None) == V.ERR_UNSUPPORTED_SHAPE  # > 8 remote maps
+    assert remote(ctypes.byref(shape), world, world, out, ws, wsb, None) == V.ERR_INVALID_ARG
+    assert remote(ctypes.byref(shape), world, -1, out, ws, wsb, None) == V.ERR_INVALID_ARG
+    assert remote(ctypes.byref(shape), world, 0, out, ws, wsb - 1, None) == V.ERR_WORKSPACE_TOO_SMALL
+    assert remote(ctypes.byref(shape), world, 0, None, ws, wsb, None) == V.ERR_INVALID_ARG
+    assert remote(ctypes.byref(shape), world, 0, out + 8, ws, wsb, None) == V.ERR_MISALIGNED
+    assert remote(ctypes.byref(shape), world, 0, ws + 256, ws, wsb, None) == V.ERR_INVALID_ARG   # out inside the workspace
