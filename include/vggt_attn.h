@@ -61,7 +61,7 @@
 extern "C" {
 #endif
 
-#define VGGT_ATTN_ABI_VERSION 3
+#define VGGT_ATTN_ABI_VERSION 4
 
 /* Return codes (0 = success). */
 enum {

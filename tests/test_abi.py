@@ -47,7 +47,7 @@ def test_library_exports_every_declared_function(V):
     lib = ctypes.CDLL(V.LIB_PATH)
     for n in names:
         assert hasattr(lib, n), n
-    assert V.vggt_attn_abi_version() == 3
+    assert V.vggt_attn_abi_version() == 4
 
 
 def test_error_strings(V):
